@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""BitLinear W1.58A8 benchmark on B200.
+
+Workload (default, "decode"): one token (M=1) through the seven BitLinear
+projections (q, k, v, o, gate, up, down) of each of the 30 layers of the
+BitNet b1.58 2B4T shapes: 210 full BitLinear forwards per step (fused RMSNorm
+with U(0.5,1.5) gain, per-token int8 quantisation, ternary matmul, rescale,
+bf16 output), 521 MB of distinct packed weights, more than the 126 MB L2, so
+every step streams them from HBM.  Inputs: x ~ N(0,1) with 0.1% outliers x20;
+weights absmean-ternarised from N(0, 0.02) masters.  tokens/s = M / step time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs its own replica (the path has no exchange step)
+and the reported value is the tokens of all ranks / the slowest rank's time.
+Prints one JSON line on rank 0.
+"""
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "BitLinear W1.58A8 tokens/s; % roofline (GEMV HBM GB/s, GEMM int8 TOPS)"
+DECODE_KERNEL_SOURCES = ("common.cuh", "quant.cuh", "decode.cuh")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--layers", type=int, default=30)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU work budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=300),
+            device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting"}
+
+    def __init__(self, index):
+        self.samples = []
+        self.reasons = 0
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # reported, never fatal
+            self.err = repr(e)
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        while not self.stop_flag.is_set():
+            self._sample()
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.stop_flag = threading.Event()
+            self._sample()
+            self.th = threading.Thread(target=self._run, daemon=True)
+            self.th.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._sample()
+            self.stop_flag.set()
+            self.th.join()
+
+    def result(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        reasons = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# the decode workload
+# ---------------------------------------------------------------------------
+def token_work_units(WL, layers):
+    """Per-projection MAC counts (work units) of one token through all layers."""
+    return sum(p.N * p.K for p in WL.PROJECTIONS) * layers
+
+
+class DecodeWorkload:
+    def __init__(self, layers, M=1):
+        import ternary_weight_bitlinear_b200 as B
+        from ternary_weight_bitlinear_b200 import workloads as WL
+        self.B, self.WL, self.M, self.layers = B, WL, M, layers
+        dev = torch.device("cuda")
+        specs = [(l, p) for l in range(layers) for p in WL.PROJECTIONS]
+        x_elems = sum(M * p.K for _, p in specs)
+        y_elems = sum(M * p.N for _, p in specs)
+        self.x_dev = torch.empty(x_elems, dtype=torch.bfloat16, device=dev)
+        self.y_dev = torch.empty(y_elems, dtype=torch.bfloat16, device=dev)
+        self.x_host = torch.empty(x_elems, dtype=torch.bfloat16).pin_memory()
+        self.y_host = torch.empty(y_elems, dtype=torch.bfloat16).pin_memory()
+        self.problems = []
+        gains = {}
+        xo = yo = 0
+        self.weight_bytes = 0
+        for l, p in specs:
+            W = torch.from_numpy(WL.master_weights(p.N, p.K, WL.master_seed(l, p.name))).to(dev)
+            P, beta = B.bitlinear_pack(W)
+            del W
+            c = WL.config2_projection(l, p.name, M)
+            xv = torch.from_numpy(c["x"].reshape(-1).view(np.int16)).view(torch.bfloat16)
+            self.x_host[xo:xo + xv.numel()].copy_(xv)
+            key = (l, p.K)
+            if key not in gains:
+                gains[key] = torch.from_numpy(c["gain"].view(np.int16)).view(torch.bfloat16).to(dev)
+            self.problems.append(dict(
+                x=self.x_dev[xo:xo + M * p.K].view(M, p.K), P=P, beta=float(beta.item()),
+                gain=gains[key], y=self.y_dev[yo:yo + M * p.N].view(M, p.N), K=p.K, N=p.N))
+            self.weight_bytes += P.numel()
+            xo += M * p.K
+            yo += M * p.N
+        self.x_dev.copy_(self.x_host)
+        torch.cuda.synchronize()
+        # algorithmic bytes of one step: packed weights + x + gain + y
+        self.step_bytes = self.weight_bytes + 2 * (x_elems + sum(p["K"] for p in self.problems)
+                                                   + y_elems)
+        self.h2d_bytes = 2 * x_elems
+        self.d2h_bytes = 2 * y_elems
+        self.launches_per_step = len(self.problems)
+
+    def step(self):
+        B, eps = self.B, self.WL.RMS_EPS
+        for q in self.problems:
+            B.bitlinear_forward(q["x"], q["P"], q["beta"], gain=q["gain"], eps=eps, out=q["y"])
+
+    def capture(self):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.step()  # eager once on the side stream (caches, attributes)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step()
+        torch.cuda.synchronize()
+
+    def replay(self):
+        self.graph.replay()
+
+
+def timed(fn, steps, warmup, world):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        fn()
+    end.record()
+    end.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(end)  # ms
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sources_hash():
+    h = hashlib.sha256()
+    for name in DECODE_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "ternary_weight_bitlinear_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(launches):
+    """Per-launch DRAM traffic from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode_gemv_2b4t_m1.md")
+    try:
+        fields = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and line.startswith("- "):
+                    k, v = line[2:].split(":", 1)
+                    fields[k.strip()] = v.strip().strip("`")
+        if fields.get("kernel_sources_sha256_16") != kernel_sources_hash():
+            return None
+        return float(fields["dram_bytes_per_step"]) / launches
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (rank 0, N=1 only)
+# ---------------------------------------------------------------------------
+def oracle_layer0_problems(WL, M=1):
+    import oracle as O
+    probs = []
+    for p in WL.PROJECTIONS:
+        Pm, beta = O.pack_master(WL.master_weights(p.N, p.K, WL.master_seed(0, p.name)))
+        c = WL.config2_projection(0, p.name, M)
+        probs.append((c, Pm, beta, p))
+    return probs
+
+
+def oracle_run(O, WL, probs, budget_s=None, per_step=None):
+    """Time O.forward over the problems; return (seconds, tokens) where tokens is
+    the fraction of one token's 30-layer work the timed calls covered."""
+    units_token = token_work_units(WL, WL.LAYERS)
+    t_total = 0.0
+    units = 0
+    i = 0
+    while True:
+        c, Pm, beta, p = probs[i % len(probs)]
+        t0 = time.perf_counter()
+        O.forward(c["x"], Pm, beta, gain=c["gain"], eps=WL.RMS_EPS, norm=True)
+        t_total += time.perf_counter() - t0
+        units += p.N * p.K
+        i += 1
+        if per_step is not None and i >= per_step:
+            break
+        if budget_s is not None and t_total >= budget_s and i >= len(probs):
+            break
+    return t_total, units / units_token
+
+
+def cpu_baseline(budget_s):
+    import oracle as O
+    from ternary_weight_bitlinear_b200 import workloads as WL
+    probs = oracle_layer0_problems(WL)
+    secs, tokens = oracle_run(O, WL, probs, budget_s=budget_s)
+    return {"value": tokens / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "layer 0's seven M=1 BitLinear forwards (same shapes, seeds and "
+                      "RMSNorm as the GPU workload), repeated for %.1f s on one host core; "
+                      "tokens = covered MACs / one token's 30-layer MACs" % secs}
+
+
+def reference_arm(args, world, rank):
+    """The oracle as the reference arm: same workload, metric and unit."""
+    if rank != 0:
+        return
+    import oracle as O
+    from ternary_weight_bitlinear_b200 import workloads as WL
+    probs = oracle_layer0_problems(WL)
+    # each step: a bounded sample (7 forwards for short runs, 1 for long ones)
+    per_step = 7 if args.steps <= 60 else 1
+    for _ in range(args.warmup):
+        oracle_run(O, WL, probs, per_step=per_step)
+    secs = 0.0
+    tokens = 0.0
+    for s in range(args.steps):
+        rot = probs[(s * per_step) % 7:] + probs[:(s * per_step) % 7]
+        t, tk = oracle_run(O, WL, rot, per_step=per_step)
+        secs += t
+        tokens += tk
+    value = tokens / secs
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * secs / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": workload_config(args, None),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": "%d oracle BitLinear forward(s) per step from layer 0's "
+                                       "seven projections, rotating" % per_step},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(args, wl):
+    cfg = {"workload": "decode M=1: one token through the 7 BitLinear projections "
+                       "(q,k,v,o 2560->2560/640, gate/up 2560->6912, down 6912->2560) of each "
+                       "of the 30 BitNet-2B4T layers; fused RMSNorm, int8 absmax, ternary "
+                       "matmul, bf16 out",
+           "M": 1, "layers": args.layers, "hidden": 2560, "intermediate": 6912,
+           "parallelism": "replicas" if args.gpus > 1 else "single",
+           "l2": "no flush: the 521 MB of packed weights per step exceed the 126 MB L2"}
+    if wl is not None:
+        cfg["packed_weight_bytes_per_step"] = wl.weight_bytes
+        cfg["algorithmic_bytes_per_step"] = wl.step_bytes
+    return cfg
+
+
+# ---------------------------------------------------------------------------
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    from __graft_entry__ import build
+    if rank == 0:
+        build()
+    barrier(world)
+    wl = DecodeWorkload(args.layers)
+    wl.capture()
+
+    # device-resident timing (CUDA graph of the 210 forwards)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ms = timed(wl.replay, args.steps, args.warmup, world)
+    ms = max_over_ranks(ms, world)
+    ms_step = ms / args.steps
+    value = world * wl.M * args.steps / (ms / 1000.0)
+
+    # end to end: pinned host x -> device, forwards, device -> pinned host y
+    def e2e_step():
+        wl.x_dev.copy_(wl.x_host, non_blocking=True)
+        wl.replay()
+        wl.y_host.copy_(wl.y_dev, non_blocking=True)
+    ms_e2e = max_over_ranks(timed(e2e_step, args.steps, args.warmup, world), world)
+    e2e_value = world * wl.M * args.steps / (ms_e2e / 1000.0)
+
+    status = wl.B.bitlinear_device_status()
+    if status != 0:
+        raise RuntimeError("device status %d after the timed region" % status)
+
+    hbm, hbm_src = measured_peaks()
+    launch_ms = ms_step / wl.launches_per_step
+    bytes_per_launch = wl.step_bytes / wl.launches_per_step
+    achieved = bytes_per_launch / (launch_ms / 1000.0) / 1e9
+    traffic = recorded_traffic(wl.launches_per_step)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "int8", "data": "synthetic", "config": workload_config(args, wl),
+                "roofline": {"bound": "hbm", "kernel": "decode_kernel (fused RMSNorm+quant+GEMV)",
+                             "achieved": achieved, "peak": hbm, "peak_source": hbm_src,
+                             "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
+                             "launch_us": launch_ms * 1000.0,
+                             "bytes_per_launch": bytes_per_launch},
+                "e2e": {"value": e2e_value, "unit": "tokens/s",
+                        "h2d_bytes_per_step": wl.h2d_bytes, "d2h_bytes_per_step": wl.d2h_bytes},
+                "gpu_launches": wl.launches_per_step * args.steps,
+                "clocks": clk.result()}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        del wl.graph
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

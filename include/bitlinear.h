@@ -1,0 +1,175 @@
+/*
+ * bitlinear.h -- C ABI of libbitlinear.so, the B200 (sm_100a) implementation of
+ * the inference-time BitLinear forward of BitNet b1.58 (ternary weights, int8
+ * activations: W1.58A8).
+ *
+ * Sources (web pages, cited by title and section):
+ *   [QG] "BitNet" -- transformers quantization guide, steps 1-3 of the recipe.
+ *   [BG] "Transformers 实战 BitNet 1.58 位量化：BitLinear 原理、量化流程与推理加载全指南",
+ *        sections "BitLinear 的三步量化" (weight / activation quantisation) and
+ *        "推理侧 BitLinear：打包权重、解包与缩放" (pack_weights, unpack_weights,
+ *        BitLinear.forward, post_quant_process).
+ *   [MD] "BitNet" -- transformers model doc, model details (W1.58A8, ReLU^2,
+ *        subln) and BitNetConfig (rms_norm_eps = 1e-5).
+ *
+ * Conventions for every entry point
+ *   - Pointers marked "device" must point to memory the current CUDA device can
+ *     read/write (cudaMalloc, torch CUDA tensors).  The caller owns all memory;
+ *     the library allocates nothing and keeps no pointer after returning.
+ *   - Row-major, contiguous tensors.  bf16 tensors are passed as uint16_t bit
+ *     patterns.  Sizes are element counts.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on that stream; results are ready when the stream is.
+ *   - Arguments are checked on the host before anything is launched; a failed
+ *     check returns its status and launches nothing.  A launch failure returns
+ *     BL_ERR_CUDA.  A kernel that stops waiting on an internal barrier after its
+ *     time limit records BL_ERR_TIMEOUT in a device status word, read back with
+ *     bitlinear_device_status().
+ *   - Shapes: M >= 0 tokens (M == 0 is a no-op returning BL_OK), K > 0 input
+ *     features with K % 16 == 0 and K <= BL_MAX_K, N > 0 output features with
+ *     N % 4 == 0.  Tensor pointers must be 16-byte aligned.
+ *   - Numerics: every floating-point step is a single IEEE operation rounded to
+ *     nearest-even, in the order written below; sums named "exact" are taken
+ *     exactly up to one final rounding to binary64 (computed in binary64 with
+ *     error-free transformations).  Codes, packed bytes and int32 accumulators
+ *     are therefore reproducible bit for bit.
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BL_ABI_VERSION 1
+#define BL_MAX_K 65536
+
+typedef enum {
+    BL_OK = 0,
+    BL_ERR_NULL = 1,      /* a required pointer is NULL */
+    BL_ERR_SHAPE = 2,     /* M/K/N outside the rules above */
+    BL_ERR_ALIGN = 3,     /* a tensor pointer is not 16-byte aligned */
+    BL_ERR_DTYPE = 4,     /* unknown output dtype, or a dtype/option mismatch */
+    BL_ERR_WORKSPACE = 5, /* workspace missing or smaller than required */
+    BL_ERR_CUDA = 6,      /* a CUDA launch or runtime call failed */
+    BL_ERR_TIMEOUT = 7,   /* a device-side bounded wait expired */
+    BL_ERR_DEVICE = 8     /* no usable sm_100 device is current */
+} bl_status;
+
+typedef enum { BL_OUT_BF16 = 0, BL_OUT_F32 = 1 } bl_out_dtype;
+
+/* Version of this ABI (BL_ABI_VERSION). */
+int bitlinear_abi_version(void);
+
+/* Static description of a status code. */
+const char* bitlinear_status_string(bl_status status);
+
+/* ---- weight preparation (offline, load time) ---------------------------- */
+
+/* Workspace needed by bitlinear_pack for an [N,K] master weight. */
+bl_status bitlinear_pack_workspace_size(int64_t N, int64_t K, size_t* bytes);
+
+/* Absmean ternarisation and 2-bit packing of a master weight ([BG] "BitLinear
+ * 的三步量化" steps 1-2, [QG] steps 1-2; packing: [BG] "推理侧 BitLinear",
+ * pack_weights).
+ *   W         device fp32 [N,K] master weight (nn.Linear layout: out x in).
+ *   P         device uint8 [N/4,K] output.  Bits 2i..2i+1 of P[r,k] hold
+ *             t[i*N/4 + r, k] + 1 in {0,1,2} ("block" layout: bit pair i is the
+ *             i-th quarter of the output rows).
+ *   beta_out  device float[1] output: beta = max(RN32(exact sum|W| / (N*K)),
+ *             1e-5), the absmean weight scale later passed to the forward.
+ *   t[n,k] = clamp(round_half_even(RN32(W[n,k] * RN32(1/beta))), -1, 1).
+ *   workspace device, >= bitlinear_pack_workspace_size(N, K) bytes. */
+bl_status bitlinear_pack(const float* W, int64_t N, int64_t K, uint8_t* P, float* beta_out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Pack already-ternary weights t[N,K] (values in {-1,0,1}, device int8) into P
+ * [N/4,K] with the layout above ([BG] pack_weights).  Values outside {-1,0,1}
+ * are not checked on the device; they produce unspecified codes. */
+bl_status bitlinear_pack_ternary(const int8_t* t, int64_t N, int64_t K, uint8_t* P,
+                                 void* stream);
+
+/* Inverse of the packing ([BG] unpack_weights: bit pair i, masked by 3 << 2i,
+ * shifted down, minus one): t[i*N/4 + r, k] = ((P[r,k] >> 2i) & 3) - 1, into
+ * device int8 t[N,K].  A bit pair 11 (never written by the packers) gives +2. */
+bl_status bitlinear_unpack(const uint8_t* P, int64_t N, int64_t K, int8_t* t, void* stream);
+
+/* ---- activation quantisation --------------------------------------------- */
+
+/* Optional RMSNorm, then per-token absmax int8 quantisation ([BG] "BitLinear
+ * 的三步量化" step 3, [QG] step 3; the norm is the optional first step of
+ * BitLinear.forward in [BG] "推理侧 BitLinear", eps from [MD] BitNetConfig).
+ *   x       device bf16 [M,K].
+ *   gain    device bf16 [K] RMSNorm weight, or NULL for no norm.
+ *   eps     RMSNorm epsilon (ignored when gain is NULL).
+ *   q       device int8 [M,K] output codes.
+ *   s_x     device fp32 [M] output multipliers.
+ *   rowsum  device int32 [M] output sum_k q[m,k], or NULL.
+ * With the norm:  r = RN32(1/sqrt(exact sum_k x^2 / K + eps)) (binary64 ops),
+ *                 h = RN32(RN32(x*r)*gain);  without it: h = x.
+ * Then s_x = RN32(127 / max(max_k |h|, 1e-5)), q = clamp(rint(RN32(h*s_x)),
+ * -128, 127).  No workspace. */
+bl_status bitlinear_act_quant(const uint16_t* x, const uint16_t* gain, float eps, int64_t M,
+                              int64_t K, int8_t* q, float* s_x, int32_t* rowsum, void* stream);
+
+/* ---- forward -------------------------------------------------------------- */
+
+/* Workspace bitlinear_forward needs for this shape (0 when none). */
+bl_status bitlinear_forward_workspace_size(int64_t M, int64_t K, int64_t N, size_t* bytes);
+
+/* The whole BitLinear forward ([BG] "推理侧 BitLinear": optional RMSNorm,
+ * unpack, activation_quant, F.linear, post_quant_process):
+ *   x      device bf16 [M,K];  gain: device bf16 [K] or NULL (no norm);  eps.
+ *   P      device uint8 [N/4,K] packed weights (bitlinear_pack layout).
+ *   beta   host float: the absmean weight scale of P.
+ *   y      device [M,N], bf16 or fp32 per y_dtype:
+ *          y = RN32(RN32(float(acc) * beta) / s_x[m]), acc = sum_k q[m,k] t[n,k]
+ *          exact in int32; rounded once more to bf16 when y_dtype is BL_OUT_BF16.
+ *   workspace  device, >= bitlinear_forward_workspace_size(M,K,N) bytes (may be
+ *          NULL when that size is 0).  Holds the int8 codes between kernels. */
+bl_status bitlinear_forward(const uint16_t* x, const uint16_t* gain, float eps,
+                            const uint8_t* P, float beta, int64_t M, int64_t K, int64_t N,
+                            void* y, bl_out_dtype y_dtype, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* Matmul and rescale on activations already quantised by bitlinear_act_quant
+ * (so several projections can share one quantisation):
+ *   q [M,K] int8, s_x [M] fp32, rowsum [M] int32 (all device, as produced by
+ *   bitlinear_act_quant with a non-NULL rowsum);  P, beta, y, y_dtype as in
+ *   bitlinear_forward.
+ *   residual  device bf16 [M,N] or NULL.  When given, y_dtype must be
+ *             BL_OUT_BF16 and y = bf16(float(residual) + float(bf16(y))) (the
+ *             residual add of a decoder block); y may alias residual. */
+bl_status bitlinear_forward_quantized(const int8_t* q, const float* s_x, const int32_t* rowsum,
+                                      const uint8_t* P, float beta, int64_t M, int64_t K,
+                                      int64_t N, void* y, bl_out_dtype y_dtype,
+                                      const uint16_t* residual, void* stream);
+
+/* The exact int32 accumulator acc[m,n] = sum_k q[m,k] t[n,k] of the same
+ * kernels, without the rescale (for bit-exact verification).  Arguments as in
+ * bitlinear_forward_quantized; acc is device int32 [M,N]. */
+bl_status bitlinear_accumulate(const int8_t* q, const int32_t* rowsum, const uint8_t* P,
+                               int64_t M, int64_t K, int64_t N, int32_t* acc, void* stream);
+
+/* ---- FFN glue ([MD] model details: ReLU^2 FFN; [BG] ffn_sub_norm) ---------- */
+
+/* z = bf16(RN32(RN32(relu(a) * relu(a)) * b)) elementwise over n values;
+ * a = gate output, b = up output, all device bf16.  z may alias a or b. */
+bl_status bitlinear_relu2_mul(const uint16_t* a, const uint16_t* b, int64_t n, uint16_t* z,
+                              void* stream);
+
+/* ---- device status -------------------------------------------------------- */
+
+/* Synchronises `stream`, then returns and clears the library's device status
+ * word on the current device: BL_OK, or BL_ERR_TIMEOUT if a kernel gave up on a
+ * bounded wait since the last call. */
+bl_status bitlinear_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

@@ -1,0 +1,11 @@
+"""B200 (sm_100a) BitLinear W1.58A8 forward of BitNet b1.58.
+
+The compute lives in ``libbitlinear.so`` (C ABI, declared in include/bitlinear.h);
+:mod:`ternary_weight_bitlinear_b200.bitlinear` is its thin ctypes binding.
+"""
+from .bitlinear import (BL_MAX_K, BL_OUT_BF16, BL_OUT_F32, BitLinearError, LIB_PATH,  # noqa: F401
+                        bitlinear_accumulate, bitlinear_act_quant, bitlinear_device_status,
+                        bitlinear_forward, bitlinear_forward_quantized,
+                        bitlinear_forward_workspace_size, bitlinear_pack,
+                        bitlinear_pack_ternary, bitlinear_pack_workspace_size,
+                        bitlinear_relu2_mul, bitlinear_unpack, lib, status_string)

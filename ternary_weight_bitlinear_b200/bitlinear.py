@@ -1,0 +1,224 @@
+"""Python binding of libbitlinear.so (ctypes): argument marshalling only.
+
+Every function has the name of the C entry point it calls and takes CUDA
+torch tensors; all arithmetic runs in the library's kernels.  There is no
+fallback: if ``libbitlinear.so`` is missing or no sm_100 device is current,
+calls raise.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbitlinear.so")
+
+BL_OUT_BF16 = 0
+BL_OUT_F32 = 1
+BL_MAX_K = 65536
+
+STATUS = {0: "BL_OK", 1: "BL_ERR_NULL", 2: "BL_ERR_SHAPE", 3: "BL_ERR_ALIGN", 4: "BL_ERR_DTYPE",
+          5: "BL_ERR_WORKSPACE", 6: "BL_ERR_CUDA", 7: "BL_ERR_TIMEOUT", 8: "BL_ERR_DEVICE"}
+
+# C signatures: name -> (argtypes, restype)
+_P, _I64, _F32, _SZ, _INT = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, \
+    ctypes.c_int
+SIGNATURES = {
+    "bitlinear_abi_version": ([], _INT),
+    "bitlinear_status_string": ([_INT], ctypes.c_char_p),
+    "bitlinear_pack_workspace_size": ([_I64, _I64, ctypes.POINTER(_SZ)], _INT),
+    "bitlinear_pack": ([_P, _I64, _I64, _P, _P, _P, _SZ, _P], _INT),
+    "bitlinear_pack_ternary": ([_P, _I64, _I64, _P, _P], _INT),
+    "bitlinear_unpack": ([_P, _I64, _I64, _P, _P], _INT),
+    "bitlinear_act_quant": ([_P, _P, _F32, _I64, _I64, _P, _P, _P, _P], _INT),
+    "bitlinear_forward_workspace_size": ([_I64, _I64, _I64, ctypes.POINTER(_SZ)], _INT),
+    "bitlinear_forward": ([_P, _P, _F32, _P, _F32, _I64, _I64, _I64, _P, _INT, _P, _SZ, _P], _INT),
+    "bitlinear_forward_quantized": ([_P, _P, _P, _P, _F32, _I64, _I64, _I64, _P, _INT, _P, _P],
+                                    _INT),
+    "bitlinear_accumulate": ([_P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
+    "bitlinear_relu2_mul": ([_P, _P, _I64, _P, _P], _INT),
+    "bitlinear_device_status": ([_P], _INT),
+}
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__("%s failed: %s (%s)" % (fn, STATUS.get(status, status),
+                                                  status_string(status)))
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libbitlinear.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libbitlinear.so is not built; run "
+                              "`python -m ternary_weight_bitlinear_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().bitlinear_status_string(status).decode()
+
+
+def _check(fn, status):
+    if status != 0:
+        raise BitLinearError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, name, ndim=None):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise TypeError("%s must be a contiguous CUDA %s tensor" % (name, dtype))
+    if ndim is not None and t.dim() != ndim:
+        raise TypeError("%s must have %d dimensions" % (name, ndim))
+    return t
+
+
+# --- sizes --------------------------------------------------------------------
+def bitlinear_pack_workspace_size(N, K):
+    n = ctypes.c_size_t()
+    _check("bitlinear_pack_workspace_size", lib().bitlinear_pack_workspace_size(N, K, ctypes.byref(n)))
+    return n.value
+
+
+def bitlinear_forward_workspace_size(M, K, N):
+    n = ctypes.c_size_t()
+    _check("bitlinear_forward_workspace_size",
+           lib().bitlinear_forward_workspace_size(M, K, N, ctypes.byref(n)))
+    return n.value
+
+
+def _workspace(nbytes, device):
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+# --- weights --------------------------------------------------------------------
+def bitlinear_pack(W, P=None, beta=None, workspace=None, stream=None):
+    """fp32 master W[N,K] -> (P uint8 [N/4,K], beta fp32 [1] on the device)."""
+    _need(W, torch.float32, "W", 2)
+    N, K = W.shape
+    P = torch.empty((N // 4, K), dtype=torch.uint8, device=W.device) if P is None else P
+    beta = torch.empty(1, dtype=torch.float32, device=W.device) if beta is None else beta
+    ws = _workspace(bitlinear_pack_workspace_size(N, K), W.device) if workspace is None else workspace
+    _check("bitlinear_pack", lib().bitlinear_pack(_ptr(W), N, K, _ptr(P), _ptr(beta), _ptr(ws),
+                                                  ws.numel(), _stream(stream)))
+    return P, beta
+
+
+def bitlinear_pack_ternary(t, P=None, stream=None):
+    _need(t, torch.int8, "t", 2)
+    N, K = t.shape
+    P = torch.empty((N // 4, K), dtype=torch.uint8, device=t.device) if P is None else P
+    _check("bitlinear_pack_ternary", lib().bitlinear_pack_ternary(_ptr(t), N, K, _ptr(P),
+                                                                  _stream(stream)))
+    return P
+
+
+def bitlinear_unpack(P, N=None, t=None, stream=None):
+    _need(P, torch.uint8, "P", 2)
+    R, K = P.shape
+    N = 4 * R if N is None else N
+    t = torch.empty((N, K), dtype=torch.int8, device=P.device) if t is None else t
+    _check("bitlinear_unpack", lib().bitlinear_unpack(_ptr(P), N, K, _ptr(t), _stream(stream)))
+    return t
+
+
+# --- activations ------------------------------------------------------------------
+def bitlinear_act_quant(x, gain=None, eps=1e-5, q=None, s_x=None, rowsum=None, stream=None):
+    """bf16 x[M,K] (+ optional RMSNorm gain) -> (q int8 [M,K], s_x fp32 [M], rowsum int32 [M])."""
+    _need(x, torch.bfloat16, "x", 2)
+    if gain is not None:
+        _need(gain, torch.bfloat16, "gain", 1)
+    M, K = x.shape
+    dev = x.device
+    q = torch.empty((M, K), dtype=torch.int8, device=dev) if q is None else q
+    s_x = torch.empty(M, dtype=torch.float32, device=dev) if s_x is None else s_x
+    rowsum = torch.empty(M, dtype=torch.int32, device=dev) if rowsum is None else rowsum
+    _check("bitlinear_act_quant", lib().bitlinear_act_quant(
+        _ptr(x), _ptr(gain), eps, M, K, _ptr(q), _ptr(s_x), _ptr(rowsum), _stream(stream)))
+    return q, s_x, rowsum
+
+
+# --- forward ----------------------------------------------------------------------
+def _out_code(dtype):
+    if dtype == torch.bfloat16:
+        return BL_OUT_BF16
+    if dtype == torch.float32:
+        return BL_OUT_F32
+    raise TypeError("output dtype must be torch.bfloat16 or torch.float32")
+
+
+def bitlinear_forward(x, P, beta, gain=None, eps=1e-5, out_dtype=torch.bfloat16, out=None,
+                      workspace=None, N=None, stream=None):
+    """Full BitLinear forward: bf16 x[M,K] -> y[M,N] (bf16 or fp32).  ``beta`` is a host float."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(P, torch.uint8, "P", 2)
+    if gain is not None:
+        _need(gain, torch.bfloat16, "gain", 1)
+    M, K = x.shape
+    N = 4 * P.shape[0] if N is None else N
+    y = torch.empty((M, N), dtype=out_dtype, device=x.device) if out is None else out
+    if workspace is None:
+        need = bitlinear_forward_workspace_size(M, K, N)
+        workspace = _workspace(need, x.device) if need else None
+    _check("bitlinear_forward", lib().bitlinear_forward(
+        _ptr(x), _ptr(gain), eps, _ptr(P), float(beta), M, K, N, _ptr(y), _out_code(y.dtype),
+        _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream)))
+    return y
+
+
+def bitlinear_forward_quantized(q, s_x, rowsum, P, beta, out_dtype=torch.bfloat16, residual=None,
+                                out=None, N=None, stream=None):
+    _need(q, torch.int8, "q", 2)
+    _need(P, torch.uint8, "P", 2)
+    M, K = q.shape
+    N = 4 * P.shape[0] if N is None else N
+    y = torch.empty((M, N), dtype=out_dtype, device=q.device) if out is None else out
+    _check("bitlinear_forward_quantized", lib().bitlinear_forward_quantized(
+        _ptr(q), _ptr(s_x), _ptr(rowsum), _ptr(P), float(beta), M, K, N, _ptr(y),
+        _out_code(y.dtype), _ptr(residual), _stream(stream)))
+    return y
+
+
+def bitlinear_accumulate(q, rowsum, P, N=None, out=None, stream=None):
+    _need(q, torch.int8, "q", 2)
+    _need(P, torch.uint8, "P", 2)
+    M, K = q.shape
+    N = 4 * P.shape[0] if N is None else N
+    acc = torch.empty((M, N), dtype=torch.int32, device=q.device) if out is None else out
+    _check("bitlinear_accumulate", lib().bitlinear_accumulate(
+        _ptr(q), _ptr(rowsum), _ptr(P), M, K, N, _ptr(acc), _stream(stream)))
+    return acc
+
+
+def bitlinear_relu2_mul(a, b, out=None, stream=None):
+    _need(a, torch.bfloat16, "a")
+    _need(b, torch.bfloat16, "b")
+    z = torch.empty_like(a) if out is None else out
+    _check("bitlinear_relu2_mul", lib().bitlinear_relu2_mul(_ptr(a), _ptr(b), a.numel(), _ptr(z),
+                                                            _stream(stream)))
+    return z
+
+
+def bitlinear_device_status(stream=None):
+    """Synchronise and return (and clear) the library's device status code."""
+    return lib().bitlinear_device_status(_stream(stream))

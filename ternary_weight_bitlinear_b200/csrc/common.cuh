@@ -1,0 +1,157 @@
+// common.cuh -- device helpers shared by the BitLinear kernels (sm_100a).
+//
+// Inline PTX for the pieces CUDA C++ does not expose directly: mbarriers,
+// bulk asynchronous copies (TMA engine, non-multicast), proxy fences,
+// programmatic dependent launch and the global timer used to bound waits.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace bl {
+
+constexpr float kScaleFloor = 1e-5f;  // clamp floor of both scales (absmean, absmax)
+
+// Device status word: bit 0 = a bounded wait expired.  Read and cleared by
+// bitlinear_device_status().
+__device__ unsigned int g_status;
+constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
+    return __uint_as_float(b << 16);
+}
+
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---- mbarrier --------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// Make barrier initialisation visible to the async proxy (bulk copies) and the
+// rest of the CTA; follow with __syncthreads().
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of the barrier to complete, for at most kWaitLimitNs.
+// On expiry records kStatusTimeout and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_status, kStatusTimeout);
+            return false;
+        }
+    }
+}
+
+// ---- bulk copies (TMA engine, no multicast) ---------------------------------
+// Global -> this CTA's shared memory; completion counted in bytes on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Same, with an L2 evict-first hint for data read exactly once (streamed weights).
+__device__ __forceinline__ void bulk_g2s_stream(uint32_t dst, const void* src, uint32_t bytes,
+                                                uint32_t bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// Order this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy accesses (a bulk copy refilling a buffer just read).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---- programmatic dependent launch -----------------------------------------
+// Block until the grids this one depends on have completed and their memory
+// is visible (no-op when launched without the PDL attribute).
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Allow the next grid in the stream to begin launching.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---- integer dot products ----------------------------------------------------
+// d = c + sum_{j<4} a.u8[j] * b.s8[j]
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// ---- error-free binary64 accumulation ----------------------------------------
+// (hi, lo) holds a running sum; add v with TwoSum so the rounding error of the
+// hi addition is carried exactly into lo.  Explicit _rn intrinsics keep the
+// compiler from contracting or reassociating.
+__device__ __forceinline__ void dd_add(double& hi, double& lo, double v) {
+    const double s = __dadd_rn(hi, v);
+    const double bv = __dsub_rn(s, hi);
+    const double av = __dsub_rn(s, bv);
+    const double e = __dadd_rn(__dsub_rn(hi, av), __dsub_rn(v, bv));
+    hi = s;
+    lo = __dadd_rn(lo, e);
+}
+
+__device__ __forceinline__ void dd_merge(double& hi, double& lo, double ohi, double olo) {
+    dd_add(hi, lo, ohi);
+    lo = __dadd_rn(lo, olo);
+}
+
+}  // namespace bl

@@ -1,0 +1,192 @@
+// quant.cuh -- optional RMSNorm + per-token absmax int8 quantisation.
+//
+// Follows the "Transformers 实战 BitNet 1.58 位量化" walkthrough, section
+// "BitLinear 的三步量化", step 3 (per-token absmax to [-128,127], scale
+// 127/max clamped at 1e-5) and the forward order of section "推理侧 BitLinear"
+// (RMSNorm first when present).  The norm formula is the standard RMSNorm with
+// the sum of squares taken exactly (binary64 with error-free TwoSum, fixed
+// reduction order), so r = RN32(1/sqrt(SS/K + eps)) is reproducible bit for bit.
+//
+// One CTA works on one token row; all loads are 16-byte vectors (8 bf16).  The
+// row is re-read from L1 in each pass instead of being staged.
+#pragma once
+
+#include "common.cuh"
+
+namespace bl {
+
+template <int NT>
+struct QuantScratch {
+    double dhi[NT / 32];
+    double dlo[NT / 32];
+    float fmax_[NT / 32];
+    int isum[NT / 32];
+    double dres;
+    float fres;
+    int ires;
+};
+
+// Deterministic block sum of (hi, lo) pairs: fixed shuffle tree inside each
+// warp, then warps merged in index order by thread 0.  Result = RN64(hi + lo).
+template <int NT>
+__device__ __forceinline__ double block_sum_dd(double hi, double lo, QuantScratch<NT>& sc) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double ohi = __shfl_down_sync(0xffffffffu, hi, o);
+        const double olo = __shfl_down_sync(0xffffffffu, lo, o);
+        dd_merge(hi, lo, ohi, olo);  // only lane 0's result is used
+    }
+    if (lane == 0) { sc.dhi[warp] = hi; sc.dlo[warp] = lo; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double h = sc.dhi[0], l = sc.dlo[0];
+        for (int w = 1; w < NT / 32; ++w) dd_merge(h, l, sc.dhi[w], sc.dlo[w]);
+        sc.dres = __dadd_rn(h, l);
+    }
+    __syncthreads();
+    return sc.dres;
+}
+
+template <int NT>
+__device__ __forceinline__ float block_max(float v, QuantScratch<NT>& sc) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) sc.fmax_[warp] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = sc.fmax_[0];
+        for (int w = 1; w < NT / 32; ++w) m = fmaxf(m, sc.fmax_[w]);
+        sc.fres = m;
+    }
+    __syncthreads();
+    return sc.fres;
+}
+
+template <int NT>
+__device__ __forceinline__ int block_sum_int(int v, QuantScratch<NT>& sc) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) sc.isum[warp] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int s = 0;
+        for (int w = 0; w < NT / 32; ++w) s += sc.isum[w];
+        sc.ires = s;
+    }
+    __syncthreads();
+    return sc.ires;
+}
+
+// Eight bf16 values of one 16-byte vector, widened to binary32 (exact).
+__device__ __forceinline__ void unpack8_bf16(const uint4 u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        f[2 * j] = bf16_bits_to_float(w[j] & 0xFFFFu);
+        f[2 * j + 1] = bf16_bits_to_float(w[j] >> 16);
+    }
+}
+
+// The normalised value h of one element: RN32(RN32(x * r) * g).
+__device__ __forceinline__ float norm_elem(float x, float r, float g) {
+    return __fmul_rn(__fmul_rn(x, r), g);
+}
+
+// Quantise one token row.  x: K bf16 (global, 16-byte aligned); gain: K bf16
+// or nullptr (no norm); q: K int8 destination (global or shared, 8-byte
+// aligned).  Every thread of the CTA must call it; s_out and rowsum_out are
+// valid in every thread on return.
+template <int NT>
+__device__ void quantize_row(const uint16_t* __restrict__ x, const uint16_t* __restrict__ gain,
+                             float eps, int K, int8_t* __restrict__ q, QuantScratch<NT>& sc,
+                             float& s_out, int& rowsum_out) {
+    const int nvec = K >> 3;
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    const uint4* gv = reinterpret_cast<const uint4*>(gain);
+    const bool norm = gain != nullptr;
+
+    float r = 1.0f;
+    float mx = 0.0f;
+    if (norm) {
+        double hi = 0.0, lo = 0.0;
+        for (int v = threadIdx.x; v < nvec; v += NT) {
+            float f[8];
+            unpack8_bf16(__ldg(xv + v), f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const double d = (double)f[j];
+                dd_add(hi, lo, __dmul_rn(d, d));  // exact square of a bf16 value
+            }
+        }
+        const double ss = block_sum_dd<NT>(hi, lo, sc);
+        const double ms = __ddiv_rn(ss, (double)K);
+        const double var = __dadd_rn(ms, (double)eps);
+        const double sd = __dsqrt_rn(var);
+        const double rd = __ddiv_rn(1.0, sd);
+        r = __double2float_rn(rd);
+        for (int v = threadIdx.x; v < nvec; v += NT) {
+            float f[8], g[8];
+            unpack8_bf16(__ldg(xv + v), f);
+            unpack8_bf16(__ldg(gv + v), g);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(norm_elem(f[j], r, g[j])));
+        }
+    } else {
+        for (int v = threadIdx.x; v < nvec; v += NT) {
+            float f[8];
+            unpack8_bf16(__ldg(xv + v), f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(f[j]));
+        }
+    }
+    const float m = block_max<NT>(mx, sc);
+    const float s = __fdiv_rn(127.0f, fmaxf(m, kScaleFloor));
+
+    int rs = 0;
+    for (int v = threadIdx.x; v < nvec; v += NT) {
+        float f[8], g[8];
+        unpack8_bf16(__ldg(xv + v), f);
+        if (norm) {
+            unpack8_bf16(__ldg(gv + v), g);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] = norm_elem(f[j], r, g[j]);
+        }
+        uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            int c = __float2int_rn(__fmul_rn(f[j], s));  // round half to even
+            c = min(max(c, -128), 127);
+            rs += c;
+            packed[j >> 2] |= (uint32_t)(c & 0xFF) << (8 * (j & 3));
+        }
+        reinterpret_cast<uint2*>(q)[v] = make_uint2(packed[0], packed[1]);
+    }
+    rowsum_out = block_sum_int<NT>(rs, sc);
+    s_out = s;
+}
+
+// bitlinear_act_quant: one CTA per token row.
+template <int NT>
+__global__ void __launch_bounds__(NT) act_quant_kernel(const uint16_t* __restrict__ x,
+                                                       const uint16_t* __restrict__ gain,
+                                                       float eps, int K,
+                                                       int8_t* __restrict__ q,
+                                                       float* __restrict__ s_x,
+                                                       int32_t* __restrict__ rowsum) {
+    __shared__ QuantScratch<NT> sc;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t m = blockIdx.x;
+    float s;
+    int rs;
+    quantize_row<NT>(x + m * K, gain, eps, K, q + m * K, sc, s, rs);
+    if (threadIdx.x == 0) {
+        s_x[m] = s;
+        if (rowsum) rowsum[m] = rs;
+    }
+}
+
+}  // namespace bl

@@ -1,0 +1,104 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from conftest import ROOT
+
+B = pytest.importorskip("ternary_weight_bitlinear_b200")
+
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+NULL = None
+P16 = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced by host checks
+P17 = ctypes.c_void_p(0x10001)
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitlinear_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    return B.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(B.bitlinear.SIGNATURES)
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.bitlinear_abi_version() == 1
+    for code in range(9):
+        assert B.status_string(code)
+    assert "unknown" in B.status_string(99)
+
+
+def test_workspace_sizes(L):
+    assert B.bitlinear_forward_workspace_size(1, 2560, 6912) == 0
+    assert B.bitlinear_forward_workspace_size(4, 6912, 2560) == 0
+    assert B.bitlinear_forward_workspace_size(0, 2560, 2560) == 0
+    big = B.bitlinear_forward_workspace_size(4096, 2560, 6912)
+    assert big >= 4096 * 2560 + 2 * 4096 * 4
+    assert B.bitlinear_pack_workspace_size(2560, 2560) > 0
+    with pytest.raises(B.BitLinearError):
+        B.bitlinear_forward_workspace_size(1, 2561, 16)
+
+
+def _fwd(L, x=P16, gain=NULL, P=P16, M=1, K=256, N=128, y=P16, dt=0, ws=NULL, wsb=0):
+    return L.bitlinear_forward(x, gain, 1e-5, P, 1.0, M, K, N, y, dt, ws, wsb, NULL)
+
+
+def test_forward_argument_checks(L):
+    assert _fwd(L, K=250) == 2          # K % 16
+    assert _fwd(L, K=0) == 2
+    assert _fwd(L, N=130) == 2          # N % 4
+    assert _fwd(L, M=-1) == 2
+    assert _fwd(L, K=65536 + 16) == 2   # > BL_MAX_K
+    assert _fwd(L, dt=7) == 4           # unknown dtype
+    assert _fwd(L, M=0, x=NULL, P=NULL, y=NULL) == 0   # empty: no-op
+    assert _fwd(L, x=NULL) == 1
+    assert _fwd(L, y=NULL) == 1
+    assert _fwd(L, x=P17) == 3
+    assert _fwd(L, gain=P17) == 3
+    assert _fwd(L, M=64, K=2560) == 5   # needs a workspace
+    assert _fwd(L, M=64, K=2560, ws=P16, wsb=16) == 5
+
+
+def test_other_entry_points_check_arguments(L):
+    assert L.bitlinear_pack(NULL, 8, 16, P16, P16, P16, 1 << 20, NULL) == 1
+    assert L.bitlinear_pack(P16, 6, 16, P16, P16, P16, 1 << 20, NULL) == 2
+    assert L.bitlinear_pack(P16, 8, 16, P16, P16, P16, 8, NULL) == 5
+    assert L.bitlinear_pack_ternary(P16, 8, 24, P16, NULL) == 2
+    assert L.bitlinear_unpack(P17, 8, 16, P16, NULL) == 3
+    assert L.bitlinear_act_quant(NULL, NULL, 1e-5, 2, 64, P16, P16, P16, NULL) == 1
+    assert L.bitlinear_act_quant(P16, NULL, 1e-5, 0, 64, NULL, NULL, NULL, NULL) == 0
+    assert L.bitlinear_forward_quantized(P16, P16, P16, P16, 1.0, 2, 64, 8, P16, 1, P16, NULL) == 4
+    assert L.bitlinear_forward_quantized(P16, P16, NULL, P16, 1.0, 2, 64, 8, P16, 0, NULL, NULL) == 1
+    assert L.bitlinear_accumulate(P16, P16, P16, 2, 64, 10, P16, NULL) == 2
+    assert L.bitlinear_relu2_mul(P16, P16, -1, P16, NULL) == 2
+    assert L.bitlinear_relu2_mul(NULL, NULL, 0, NULL, NULL) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_no_device_is_reported_not_faked(L):
+    # valid arguments, but no CUDA device: the library refuses, it never falls back
+    assert _fwd(L) == 8
+    assert L.bitlinear_act_quant(P16, NULL, 1e-5, 2, 64, P16, P16, P16, NULL) == 8
+    assert L.bitlinear_device_status(NULL) == 8
+
+
+def test_binding_rejects_cpu_tensors():
+    x = torch.zeros(1, 256, dtype=torch.bfloat16)
+    P = torch.zeros(32, 256, dtype=torch.uint8)
+    with pytest.raises(TypeError):
+        B.bitlinear_forward(x, P, 1.0)

@@ -1,0 +1,249 @@
+"""GPU vs oracle parity, through the C ABI, on the seeded workloads.
+
+Bit-exact: packed bytes, beta, int8 codes, s_x, row sums, int32 accumulators.
+Outputs: bit-exact and within the stated tolerances (fp32 1e-6, bf16 8e-3 rel).
+Every input comes from the seeded generators; each side prepares its own
+weights from the same fp32 masters.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import ternary_weight_bitlinear_b200 as B
+from ternary_weight_bitlinear_b200 import workloads as WL
+from gpu_util import (assert_bf16_output, assert_exact, assert_f32_output, bf16_dev, bf16_host)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device_status_clean():
+    yield
+    assert B.bitlinear_device_status() == 0
+
+
+def both_pack(W):
+    """(P_gpu, beta_gpu_float, P_oracle, beta_oracle) after checking they agree."""
+    P_d, beta_d = B.bitlinear_pack(torch.from_numpy(W).cuda())
+    P_o, beta_o = O.pack_master(W)
+    beta_g = float(beta_d.item())
+    assert np.float32(beta_g) == np.float32(beta_o), (beta_g, beta_o)
+    assert_exact(P_d.cpu().numpy(), P_o, "packed bytes")
+    return P_d, beta_g, P_o, beta_o
+
+
+def run_forward(cfg, P_d, beta, P_o, beta_o, what):
+    x = cfg["x"]
+    gain = cfg.get("gain") if cfg["norm"] else None
+    out_dtype = torch.float32 if cfg["out"] == "f32" else torch.bfloat16
+    y = B.bitlinear_forward(bf16_dev(x), P_d, beta, gain=None if gain is None else bf16_dev(gain),
+                            eps=WL.RMS_EPS, out_dtype=out_dtype)
+    ref = O.forward(x, P_o, beta_o, gain=gain, eps=WL.RMS_EPS, norm=cfg["norm"])
+    if out_dtype == torch.float32:
+        assert_f32_output(y.cpu().numpy(), ref["y"], what)
+    else:
+        assert_bf16_output(bf16_host(y), O.f32_to_bf16(ref["y"]), what)
+    return y, ref
+
+
+# ---------------------------------------------------------------------------
+# weight preparation
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N,K", [(4, 16), (12, 48), (128, 256), (132, 80), (640, 2560),
+                                 (2560, 6912), (6912, 2560)])
+def test_pack_matches_oracle(N, K):
+    both_pack(WL.master_weights(N, K, seed=N * 7 + K))
+
+
+def test_pack_special_weights():
+    both_pack(np.zeros((8, 32), np.float32))                       # beta floors at 1e-5
+    both_pack(np.eye(256, dtype=np.float32))                       # t = I
+    W = WL.master_weights(64, 64, seed=3)
+    W[::3] *= 1e-20                                               # tiny magnitudes mixed in
+    both_pack(W)
+    both_pack(np.full((16, 32), 0.5, np.float32) * np.sign(WL.master_weights(16, 32, 4)))
+
+
+@pytest.mark.parametrize("N,K", [(4, 16), (36, 64), (640, 2560)])
+def test_pack_ternary_and_unpack(N, K):
+    rng = np.random.default_rng(N + K)
+    t = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    P_d = B.bitlinear_pack_ternary(torch.from_numpy(t).cuda())
+    assert_exact(P_d.cpu().numpy(), O.pack(t), "pack_ternary")
+    assert_exact(B.bitlinear_unpack(P_d).cpu().numpy(), t, "unpack")
+    # the never-written bit pair 11 decodes to +2 on both sides
+    P_bad = rng.integers(0, 256, (N // 4, K)).astype(np.uint8)
+    assert_exact(B.bitlinear_unpack(torch.from_numpy(P_bad).cuda()).cpu().numpy(),
+                 O.unpack(P_bad), "unpack of arbitrary bytes")
+
+
+# ---------------------------------------------------------------------------
+# activation quantisation
+# ---------------------------------------------------------------------------
+def special_rows(x):
+    """Overwrite a few rows with the method's degenerate cases."""
+    M, K = x.shape
+    f = WL.to_bf16_bits
+    if M > 1:
+        x[1] = 0                                                    # all zero: 1e-5 floor
+    if M > 2:
+        x[2] = f(np.full(K, 3e-7, np.float32))                      # below the floor
+    if M > 3:
+        x[3] = f(np.full(K, -2.5, np.float32))                      # constant row
+    if M > 4:
+        r = np.zeros(K, np.float32)
+        r[K // 2] = 1000.0
+        x[4] = f(r)                                                 # single spike
+    return x
+
+
+@pytest.mark.parametrize("norm", [False, True])
+@pytest.mark.parametrize("M,K", [(1, 16), (3, 256), (4, 2560), (7, 6912), (64, 2560), (257, 272)])
+def test_act_quant_matches_oracle(M, K, norm):
+    x = special_rows(WL.activations(M, K, seed=M * 131 + K, outlier_frac=0.001))
+    gain = WL.gain(K, seed=K) if norm else None
+    q, s, rs = B.bitlinear_act_quant(bf16_dev(x), None if gain is None else bf16_dev(gain),
+                                     WL.RMS_EPS)
+    q_o, s_o, rs_o = O.quantize_input(x, gain, WL.RMS_EPS, norm=norm)
+    assert_exact(s.cpu().numpy().view(np.uint32), s_o.view(np.uint32), "s_x")
+    assert_exact(q.cpu().numpy(), q_o, "codes")
+    assert_exact(rs.cpu().numpy(), rs_o, "row sums")
+
+
+# ---------------------------------------------------------------------------
+# exact int32 accumulators
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("M,K,N", [(1, 16, 4), (2, 64, 12), (3, 256, 128), (4, 2560, 640),
+                                   (5, 272, 36), (9, 6912, 2560), (1, 65536, 8), (2, 65536, 8)])
+def test_accumulate_is_exact(M, K, N):
+    x = special_rows(WL.activations(M, K, seed=M + K + N, row_std=(0.1, 10.0)))
+    W = WL.master_weights(N, K, seed=K + N)
+    P_d, beta, P_o, beta_o = both_pack(W)
+    q, s, rs = B.bitlinear_act_quant(bf16_dev(x))
+    q_o, s_o, rs_o = O.quantize_input(x)
+    assert_exact(q.cpu().numpy(), q_o, "codes")
+    acc = B.bitlinear_accumulate(q, rs, P_d)
+    acc_o = O.ternary_matmul(q_o, O.unpack(P_o))
+    assert_exact(acc.cpu().numpy(), acc_o, "int32 accumulators")
+
+
+# ---------------------------------------------------------------------------
+# the five workloads
+# ---------------------------------------------------------------------------
+def test_config1_single_bitlinear_fp32():
+    c = WL.config1()
+    P_d, beta, P_o, beta_o = both_pack(c["W"])
+    y, ref = run_forward(c, P_d, beta, P_o, beta_o, "config 1")
+    assert not y[1].any()                      # the all-zero token gives +0 outputs
+    assert not torch.signbit(y[1]).any()
+
+
+@pytest.mark.parametrize("layer", [0, 29])
+def test_config2_decode_all_projections(layer):
+    for p in WL.PROJECTIONS:
+        c = WL.config2_projection(layer, p.name)
+        W = WL.master_weights(p.N, p.K, WL.master_seed(layer, p.name))
+        P_d, beta, P_o, beta_o = both_pack(W)
+        run_forward(c, P_d, beta, P_o, beta_o, "config 2 %s" % p.name)
+
+
+@pytest.mark.parametrize("M", [8, 32, 64])
+def test_config3_batched_decode(M):
+    for p in WL.PROJECTIONS:
+        c = WL.config3_projection(0, p.name, M)
+        W = WL.master_weights(p.N, p.K, WL.master_seed(0, p.name))
+        P_d, beta, P_o, beta_o = both_pack(W)
+        run_forward(c, P_d, beta, P_o, beta_o, "config 3 %s M=%d" % (p.name, M))
+
+
+def test_config4_prefill_sampled_rows():
+    """M=4096: the GPU computes every row; the oracle recomputes a sample of
+    rows (rows are independent) and the full int8 codes of one projection."""
+    rng = np.random.default_rng(4096)
+    for name in WL.CONFIG4_PROJECTIONS:
+        c = WL.config4_projection(name)
+        p = WL.PROJECTIONS[WL.PROJ_INDEX[name]]
+        W = WL.master_weights(p.N, p.K, WL.master_seed(0, name))
+        P_d, beta, P_o, beta_o = both_pack(W)
+        x_d, g_d = bf16_dev(c["x"]), bf16_dev(c["gain"])
+        y = bf16_host(B.bitlinear_forward(x_d, P_d, beta, gain=g_d, eps=WL.RMS_EPS))
+        rows = np.unique(np.concatenate([[0, 1, 4095], rng.integers(0, 4096, 29)]))
+        ref = O.forward(c["x"][rows], P_o, beta_o, gain=c["gain"], eps=WL.RMS_EPS, norm=True)
+        assert_bf16_output(y[rows], O.f32_to_bf16(ref["y"]), "config 4 %s" % name)
+        if name == "down":
+            q, s, _ = B.bitlinear_act_quant(x_d, g_d, WL.RMS_EPS)
+            q_o, s_o, _ = O.quantize_input(c["x"], c["gain"], WL.RMS_EPS, norm=True)
+            assert_exact(q.cpu().numpy(), q_o, "config 4 codes")
+            assert_exact(s.cpu().numpy().view(np.uint32), s_o.view(np.uint32), "config 4 s_x")
+
+
+def gpu_ffn_block(x_d, g_in, g_sub, Pg, bg, Pu, bu, Pd, bd):
+    """One FFN block through the C ABI; updates x_d in place."""
+    q, s, rs = B.bitlinear_act_quant(x_d, g_in, WL.RMS_EPS)
+    a = B.bitlinear_forward_quantized(q, s, rs, Pg, bg)
+    b = B.bitlinear_forward_quantized(q, s, rs, Pu, bu)
+    z = B.bitlinear_relu2_mul(a, b)
+    q2, s2, rs2 = B.bitlinear_act_quant(z, g_sub, WL.RMS_EPS)
+    B.bitlinear_forward_quantized(q2, s2, rs2, Pd, bd, residual=x_d, out=x_d)
+    return x_d
+
+
+def test_config5_ffn_chain_30_layers():
+    M = 16
+    x = WL.config5_input(M)
+    x_d = bf16_dev(x)
+    x_o = x.copy()
+    for layer in range(WL.LAYERS):
+        L = WL.config5_layer(layer)
+        Pg, bg, Pg_o, bg_o = both_pack(L["W_gate"])
+        Pu, bu, Pu_o, bu_o = both_pack(L["W_up"])
+        Pd, bd, Pd_o, bd_o = both_pack(L["W_down"])
+        gpu_ffn_block(x_d, bf16_dev(L["g_in"]), bf16_dev(L["g_sub"]), Pg, bg, Pu, bu, Pd, bd)
+        x_o = O.ffn_block(x_o, L["g_in"], L["g_sub"], WL.RMS_EPS, Pg_o, bg_o, Pu_o, bu_o, Pd_o,
+                          bd_o)
+        assert_bf16_output(bf16_host(x_d), x_o, "config 5 after layer %d" % layer)
+
+
+# ---------------------------------------------------------------------------
+# glue and edge cases
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("n", [8, 13, 6912 * 16, 1000003])
+def test_relu2_mul_matches_oracle(n):
+    rng = np.random.default_rng(n)
+    a = WL.to_bf16_bits((rng.standard_normal(n) * 3).astype(np.float32))
+    b = WL.to_bf16_bits((rng.standard_normal(n) * 3).astype(np.float32))
+    z = B.bitlinear_relu2_mul(bf16_dev(a), bf16_dev(b))
+    assert_exact(bf16_host(z), O.relu2_mul(a, b), "relu2_mul")
+
+
+def test_residual_epilogue_matches_oracle():
+    M, K, N = 6, 256, 64
+    x = WL.activations(M, K, seed=77)
+    res = WL.activations(M, N, seed=78)
+    W = WL.master_weights(N, K, seed=79)
+    P_d, beta, P_o, beta_o = both_pack(W)
+    q, s, rs = B.bitlinear_act_quant(bf16_dev(x))
+    r_d = bf16_dev(res)
+    B.bitlinear_forward_quantized(q, s, rs, P_d, beta, residual=r_d, out=r_d)
+    y_o = O.forward(x, P_o, beta_o)["y"]
+    assert_exact(bf16_host(r_d), O.residual_add(res, O.f32_to_bf16(y_o)), "residual epilogue")
+
+
+def test_empty_batch_is_a_no_op():
+    P = torch.zeros(8, 64, dtype=torch.uint8, device="cuda")
+    x = torch.zeros(0, 64, dtype=torch.bfloat16, device="cuda")
+    y = B.bitlinear_forward(x, P, 1.0)
+    assert y.shape == (0, 32)
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 16, 4), (2, 32, 8), (3, 4096 + 16, 12), (4, 16384, 20),
+                                   (5, 64, 4), (1, 65536, 16), (3, 65536, 8)])
+def test_ragged_and_extreme_shapes(M, K, N):
+    x = WL.activations(M, K, seed=M * K + N, outlier_frac=0.01)
+    g = WL.gain(K, seed=N)
+    W = WL.master_weights(N, K, seed=K - N)
+    P_d, beta, P_o, beta_o = both_pack(W)
+    for norm in (False, True):
+        c = dict(x=x, gain=g, norm=norm, out="f32")
+        run_forward(c, P_d, beta, P_o, beta_o, "M=%d K=%d N=%d norm=%s" % (M, K, N, norm))
