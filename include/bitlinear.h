@@ -67,6 +67,11 @@ int bitlinear_abi_version(void);
 /* Static description of a status code. */
 const char* bitlinear_status_string(bl_status status);
 
+/* Text of the CUDA error behind the most recent BL_ERR_CUDA returned on the
+ * calling thread (empty if none).  Owned by the library; valid until the next
+ * call on this thread. */
+const char* bitlinear_last_error(void);
+
 /* ---- weight preparation (offline, load time) ---------------------------- */
 
 /* Workspace needed by bitlinear_pack for an [N,K] master weight. */

@@ -26,6 +26,7 @@ _P, _I64, _F32, _SZ, _INT = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, cty
 SIGNATURES = {
     "bitlinear_abi_version": ([], _INT),
     "bitlinear_status_string": ([_INT], ctypes.c_char_p),
+    "bitlinear_last_error": ([], ctypes.c_char_p),
     "bitlinear_pack_workspace_size": ([_I64, _I64, ctypes.POINTER(_SZ)], _INT),
     "bitlinear_pack": ([_P, _I64, _I64, _P, _P, _P, _SZ, _P], _INT),
     "bitlinear_pack_ternary": ([_P, _I64, _I64, _P, _P], _INT),
@@ -44,8 +45,10 @@ SIGNATURES = {
 class BitLinearError(RuntimeError):
     def __init__(self, fn, status):
         self.status = status
-        super().__init__("%s failed: %s (%s)" % (fn, STATUS.get(status, status),
-                                                  status_string(status)))
+        detail = lib().bitlinear_last_error().decode() if status == 6 else ""
+        super().__init__("%s failed: %s (%s)%s" % (fn, STATUS.get(status, status),
+                                                    status_string(status),
+                                                    " -- " + detail if detail else ""))
 
 
 _lib = None

@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <climits>
+#include <cstdio>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -55,25 +56,41 @@ bl_status current_device(int* dev, DeviceInfo* info) {
     return info->major == 10 ? BL_OK : BL_ERR_DEVICE;
 }
 
-// Opt a kernel in to the device's full dynamic shared memory (once per device)
-// and return how many of its CTAs fit on one SM with `smem` bytes.
+thread_local char g_last_error[256] = "";
+
+void record_cuda_error(cudaError_t e, const char* where) {
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", where, cudaGetErrorName(e),
+             cudaGetErrorString(e));
+}
+
+// Opt a kernel in to all the dynamic shared memory the device allows next to
+// its static shared memory (once per device) and return how many of its CTAs
+// fit on one SM with `smem` dynamic bytes; -1 on a CUDA error.
 int prepare_kernel(const void* fn, int dev, const DeviceInfo& info, int threads, int64_t smem) {
     static std::map<std::tuple<const void*, int, int64_t>, int> occ;
-    static std::map<std::pair<const void*, int>, bool> opted;
+    static std::map<std::pair<const void*, int>, int64_t> max_dyn;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!opted[{fn, dev}]) {
-        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, info.smem_optin);
-        opted[{fn, dev}] = true;
+    auto mk = std::make_pair(fn, dev);
+    if (!max_dyn.count(mk)) {
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+        if (e != cudaSuccess) { record_cuda_error(e, "cudaFuncGetAttributes"); cudaGetLastError(); return -1; }
+        const int64_t dyn = (int64_t)info.smem_optin - (int64_t)fa.sharedSizeBytes;
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+        if (e != cudaSuccess) { record_cuda_error(e, "cudaFuncSetAttribute"); cudaGetLastError(); return -1; }
+        max_dyn[mk] = dyn;
+    }
+    if (smem > max_dyn[mk]) {
+        snprintf(g_last_error, sizeof g_last_error, "kernel needs %lld B of shared memory, %lld allowed",
+                 (long long)smem, (long long)max_dyn[mk]);
+        return -1;
     }
     auto key = std::make_tuple(fn, dev, smem);
     auto it = occ.find(key);
     if (it != occ.end()) return it->second;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, (size_t)smem) !=
-        cudaSuccess) {
-        cudaGetLastError();
-        n = 1;
-    }
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, (size_t)smem);
+    if (e != cudaSuccess) { record_cuda_error(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor"); cudaGetLastError(); return -1; }
     n = std::max(n, 1);
     occ[key] = n;
     return n;
@@ -96,7 +113,11 @@ bl_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-    if (e != cudaSuccess) { cudaGetLastError(); return BL_ERR_CUDA; }
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "cudaLaunchKernelEx");
+        cudaGetLastError();
+        return BL_ERR_CUDA;
+    }
     return BL_OK;
 }
 
@@ -122,6 +143,7 @@ bl_status launch_decode_mt(const DecodeArgs& a, int dev, const DeviceInfo& info,
     auto fn = decode_kernel<MT, EPI, FUSED>;
     const int per_sm = prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, kDecThreads,
                                       smem);
+    if (per_sm < 0) return BL_ERR_CUDA;
     const int64_t grid = std::min<int64_t>(a.R, (int64_t)info.sms * per_sm);
     return launch(fn, dim3((unsigned)grid), dim3(kDecThreads), (size_t)smem, stream, a);
 }
@@ -189,6 +211,8 @@ int epi_of(bl_out_dtype d) {
 extern "C" {
 
 int bitlinear_abi_version(void) { return BL_ABI_VERSION; }
+
+const char* bitlinear_last_error(void) { return g_last_error; }
 
 const char* bitlinear_status_string(bl_status s) {
     switch (s) {
@@ -387,7 +411,9 @@ bl_status bitlinear_device_status(void* stream) {
     DeviceInfo info;
     bl_status st;
     if ((st = current_device(&dev, &info)) != BL_OK) return st;
-    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "cudaStreamSynchronize");
         cudaGetLastError();
         return BL_ERR_CUDA;
     }
