@@ -159,6 +159,34 @@ bl_status bitlinear_forward_quantized(const int8_t* q, const float* s_x, const i
 bl_status bitlinear_accumulate(const int8_t* q, const int32_t* rowsum, const uint8_t* P,
                                int64_t M, int64_t K, int64_t N, int32_t* acc, void* stream);
 
+/* ---- forward without any caller-provided memory besides inputs and outputs -- */
+
+/* Size of the library's fixed device scratch used by bitlinear_forward_noalloc. */
+#define BL_NOALLOC_SCRATCH_BYTES (2u << 20)
+
+/* Same computation and result as bitlinear_forward, for callers that cannot
+ * allocate device memory: code running while a CUDA graph is being captured
+ * (cudaMalloc is not allowed there), latency-critical loops that must not pay
+ * cudaMalloc/cudaFree's implicit device synchronisation, and plugins embedded
+ * in an engine that owns every allocation itself.  (The method's own pages
+ * have no counterpart; this is an interface convenience.)
+ *   Arguments as in bitlinear_forward, without the workspace.
+ *   Scratch: instead of a caller workspace it uses one file-scope device array
+ *   of BL_NOALLOC_SCRATCH_BYTES that every GPU which loads the library keeps
+ *   until the process exits.  The first call on a device looks up that array's
+ *   device address (so make that first call before any stream capture).
+ *   Shapes whose workspace (bitlinear_forward_workspace_size) exceeds the
+ *   array are rejected with BL_ERR_WORKSPACE before anything is launched, and
+ *   bitlinear_last_error() names both sizes.
+ *   All calls share the one array: calls that can overlap on the GPU (other
+ *   streams, other host threads) race on it and must be serialised by the
+ *   caller.  Nothing in it needs to start at zero: every byte a call reads was
+ *   written earlier in the same call.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+bl_status bitlinear_forward_noalloc(const uint16_t* x, const uint16_t* gain, float eps,
+                                    const uint8_t* P, float beta, int64_t M, int64_t K,
+                                    int64_t N, void* y, bl_out_dtype y_dtype, void* stream);
+
 /* ---- FFN glue ([MD] model details: ReLU^2 FFN; [BG] ffn_sub_norm) ---------- */
 
 /* z = bf16(RN32(RN32(relu(a) * relu(a)) * b)) elementwise over n values;

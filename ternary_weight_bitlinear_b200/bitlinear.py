@@ -38,6 +38,7 @@ SIGNATURES = {
                                     _INT),
     "bitlinear_accumulate": ([_P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "bitlinear_relu2_mul": ([_P, _P, _I64, _P, _P], _INT),
+    "bitlinear_forward_noalloc": ([_P, _P, _F32, _P, _F32, _I64, _I64, _I64, _P, _INT, _P], _INT),
     "bitlinear_device_status": ([_P], _INT),
 }
 

@@ -205,6 +205,30 @@ int epi_of(bl_out_dtype d) {
     return d == BL_OUT_BF16 ? kEpiBF16 : d == BL_OUT_F32 ? kEpiF32 : -1;
 }
 
+
+// ---- fixed scratch for bitlinear_forward_noalloc ----------------------------
+// One array per device, allocated with the module; its device address is
+// looked up once per device.  (The name is a host-side stand-in in host code:
+// only the looked-up address may be given to kernels.)
+static __device__ __align__(256) uint8_t g_noalloc_scratch[BL_NOALLOC_SCRATCH_BYTES];
+
+bl_status noalloc_scratch(int dev, void** ptr) {
+    static void* addr[64] = {};
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) {
+            record_cuda_error(e, "cudaGetSymbolAddress");
+            cudaGetLastError();
+            return BL_ERR_CUDA;
+        }
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return BL_OK;
+}
+
 }  // namespace
 
 // =============================================================================
@@ -424,6 +448,30 @@ bl_status bitlinear_device_status(void* stream) {
         return BL_ERR_CUDA;
     }
     return (v & kStatusTimeout) ? BL_ERR_TIMEOUT : BL_OK;
+}
+
+bl_status bitlinear_forward_noalloc(const uint16_t* x, const uint16_t* gain, float eps,
+                                    const uint8_t* P, float beta, int64_t M, int64_t K,
+                                    int64_t N, void* y, bl_out_dtype y_dtype, void* stream) {
+    size_t need = 0;
+    bl_status st = bitlinear_forward_workspace_size(M, K, N, &need);
+    if (st != BL_OK) return st;
+    if (need > BL_NOALLOC_SCRATCH_BYTES) {
+        snprintf(g_last_error, sizeof g_last_error,
+                 "bitlinear_forward_noalloc: this shape needs %zu bytes of scratch; the fixed "
+                 "scratch holds %u",
+                 need, (unsigned)BL_NOALLOC_SCRATCH_BYTES);
+        return BL_ERR_WORKSPACE;
+    }
+    void* scratch = nullptr;
+    if (need > 0) {
+        int dev;
+        DeviceInfo info;
+        if ((st = current_device(&dev, &info)) != BL_OK) return st;
+        if ((st = noalloc_scratch(dev, &scratch)) != BL_OK) return st;
+    }
+    return bitlinear_forward(x, gain, eps, P, beta, M, K, N, y, y_dtype, scratch,
+                             need > 0 ? (size_t)BL_NOALLOC_SCRATCH_BYTES : 0, stream);
 }
 
 }  // extern "C"
