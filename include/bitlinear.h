@@ -46,6 +46,7 @@ extern "C" {
 
 #define BL_ABI_VERSION 1
 #define BL_MAX_K 65536
+#define BL_MAX_BATCH 256
 
 typedef enum {
     BL_OK = 0,
@@ -122,7 +123,8 @@ bl_status bitlinear_act_quant(const uint16_t* x, const uint16_t* gain, float eps
 
 /* ---- forward -------------------------------------------------------------- */
 
-/* Workspace bitlinear_forward needs for this shape (0 when none). */
+/* Workspace bitlinear_forward needs for this shape: the int8 codes, s_x and
+ * row sums of the quantised activations (0 when M == 0). */
 bl_status bitlinear_forward_workspace_size(int64_t M, int64_t K, int64_t N, size_t* bytes);
 
 /* The whole BitLinear forward ([BG] "推理侧 BitLinear": optional RMSNorm,
@@ -139,6 +141,56 @@ bl_status bitlinear_forward(const uint16_t* x, const uint16_t* gain, float eps,
                             const uint8_t* P, float beta, int64_t M, int64_t K, int64_t N,
                             void* y, bl_out_dtype y_dtype, void* workspace,
                             size_t workspace_bytes, void* stream);
+
+/* One independent BitLinear problem of a batch (all pointers device). */
+typedef struct {
+    const uint16_t* x;        /* bf16 [M,K] input */
+    const uint16_t* gain;     /* bf16 [K] RMSNorm weight, or NULL for no norm */
+    const uint8_t* P;         /* uint8 [N/4,K] packed weights */
+    void* y;                  /* [M,N] output, bf16 or fp32 per y_dtype */
+    const uint16_t* residual; /* bf16 [M,N] added after the bf16 rounding, or NULL */
+    int64_t K;
+    int64_t N;
+    float beta;               /* absmean weight scale of P */
+    bl_out_dtype y_dtype;     /* BL_OUT_BF16 is required with a residual */
+} bl_problem;
+
+/* Workspace bitlinear_forward_batch needs: the sum over problems of
+ * bitlinear_forward_workspace_size(M, K, N). */
+bl_status bitlinear_forward_batch_workspace_size(const bl_problem* problems, int count, int64_t M,
+                                                 size_t* bytes);
+
+/* `count` (1..BL_MAX_BATCH) independent BitLinear forwards with the same
+ * token count M and RMSNorm eps, each exactly as bitlinear_forward computes it
+ * (plus the optional residual of bitlinear_forward_quantized; y may alias the
+ * residual).  For M <= 4 (decode) all problems' activations are quantised by
+ * one launch and all weights are streamed by one more, so a whole layer's
+ * projections cost two launches.  `problems` is a host array read during the
+ * call only.  workspace: device, >= bitlinear_forward_batch_workspace_size. */
+bl_status bitlinear_forward_batch(const bl_problem* problems, int count, int64_t M, float eps,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* One matmul problem on already-quantised activations (all pointers device;
+ * q, s_x, rowsum as produced by bitlinear_act_quant with a non-NULL rowsum). */
+typedef struct {
+    const int8_t* q;          /* int8 [M,K] codes */
+    const float* s_x;         /* fp32 [M] */
+    const int32_t* rowsum;    /* int32 [M] */
+    const uint8_t* P;         /* uint8 [N/4,K] packed weights */
+    void* y;                  /* [M,N] output, bf16 or fp32 per y_dtype */
+    const uint16_t* residual; /* bf16 [M,N] or NULL (BL_OUT_BF16 only) */
+    int64_t K;
+    int64_t N;
+    float beta;
+    bl_out_dtype y_dtype;
+} bl_quantized_problem;
+
+/* `count` (1..BL_MAX_BATCH) independent bitlinear_forward_quantized problems
+ * with the same M.  Problems may share q (projections of one input, e.g. the
+ * q|k|v or gate|up projections of a decoder layer).  For M <= 4 one launch
+ * streams every problem's weights once.  No workspace. */
+bl_status bitlinear_forward_quantized_batch(const bl_quantized_problem* problems, int count,
+                                            int64_t M, void* stream);
 
 /* Matmul and rescale on activations already quantised by bitlinear_act_quant
  * (so several projections can share one quantisation):

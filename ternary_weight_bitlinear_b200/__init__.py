@@ -5,7 +5,10 @@ The compute lives in ``libbitlinear.so`` (C ABI, declared in include/bitlinear.h
 """
 from .bitlinear import (BL_MAX_K, BL_OUT_BF16, BL_OUT_F32, BitLinearError, LIB_PATH,  # noqa: F401
                         bitlinear_accumulate, bitlinear_act_quant, bitlinear_device_status,
-                        bitlinear_forward, bitlinear_forward_quantized,
+                        bitlinear_forward, bitlinear_forward_batch,
+                        bitlinear_forward_batch_workspace_size, bitlinear_forward_quantized,
+                        bitlinear_forward_quantized_batch, make_batch,
+                        make_quantized_batch,
                         bitlinear_forward_workspace_size, bitlinear_pack,
                         bitlinear_pack_ternary, bitlinear_pack_workspace_size,
                         bitlinear_relu2_mul, bitlinear_unpack, lib, status_string)

@@ -40,7 +40,22 @@ SIGNATURES = {
     "bitlinear_relu2_mul": ([_P, _P, _I64, _P, _P], _INT),
     "bitlinear_forward_noalloc": ([_P, _P, _F32, _P, _F32, _I64, _I64, _I64, _P, _INT, _P], _INT),
     "bitlinear_device_status": ([_P], _INT),
+    "bitlinear_forward_batch_workspace_size": ([_P, _INT, _I64, ctypes.POINTER(_SZ)], _INT),
+    "bitlinear_forward_batch": ([_P, _INT, _I64, _F32, _P, _SZ, _P], _INT),
+    "bitlinear_forward_quantized_batch": ([_P, _INT, _I64, _P], _INT),
 }
+
+
+class Problem(ctypes.Structure):
+    """bl_problem: one independent BitLinear forward of a batch."""
+    _fields_ = [("x", _P), ("gain", _P), ("P", _P), ("y", _P), ("residual", _P),
+                ("K", _I64), ("N", _I64), ("beta", _F32), ("y_dtype", _INT)]
+
+
+class QuantizedProblem(ctypes.Structure):
+    """bl_quantized_problem: one matmul on already-quantised activations."""
+    _fields_ = [("q", _P), ("s_x", _P), ("rowsum", _P), ("P", _P), ("y", _P), ("residual", _P),
+                ("K", _I64), ("N", _I64), ("beta", _F32), ("y_dtype", _INT)]
 
 
 class BitLinearError(RuntimeError):
@@ -188,6 +203,59 @@ def bitlinear_forward(x, P, beta, gain=None, eps=1e-5, out_dtype=torch.bfloat16,
         _ptr(x), _ptr(gain), eps, _ptr(P), float(beta), M, K, N, _ptr(y), _out_code(y.dtype),
         _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream)))
     return y
+
+
+def make_batch(items):
+    """Build a bl_problem array from dicts with keys x, P, beta, y and optional
+    gain, residual (all CUDA tensors except the float beta)."""
+    arr = (Problem * len(items))()
+    for i, it in enumerate(items):
+        x, P, y = it["x"], it["P"], it["y"]
+        _need(x, torch.bfloat16, "x", 2)
+        _need(P, torch.uint8, "P", 2)
+        arr[i] = Problem(x.data_ptr(), _addr(it.get("gain")), P.data_ptr(), y.data_ptr(),
+                         _addr(it.get("residual")), x.shape[1], y.shape[1], float(it["beta"]),
+                         _out_code(y.dtype))
+    return arr
+
+
+def _addr(t):
+    return None if t is None else t.data_ptr()
+
+
+def bitlinear_forward_batch_workspace_size(batch, M):
+    n = ctypes.c_size_t()
+    _check("bitlinear_forward_batch_workspace_size", lib().bitlinear_forward_batch_workspace_size(
+        ctypes.cast(batch, _P), len(batch), M, ctypes.byref(n)))
+    return n.value
+
+
+def bitlinear_forward_batch(batch, M, eps=1e-5, workspace=None, stream=None):
+    """Run a bl_problem array (see make_batch) of independent forwards with M tokens each."""
+    if workspace is None:
+        workspace = _workspace(bitlinear_forward_batch_workspace_size(batch, M), "cuda")
+    _check("bitlinear_forward_batch", lib().bitlinear_forward_batch(
+        ctypes.cast(batch, _P), len(batch), M, eps, _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+
+
+def make_quantized_batch(items):
+    """Build a bl_quantized_problem array from dicts with keys q, s_x, rowsum, P,
+    beta, y and optional residual."""
+    arr = (QuantizedProblem * len(items))()
+    for i, it in enumerate(items):
+        q, P, y = it["q"], it["P"], it["y"]
+        _need(q, torch.int8, "q", 2)
+        _need(P, torch.uint8, "P", 2)
+        arr[i] = QuantizedProblem(q.data_ptr(), it["s_x"].data_ptr(), it["rowsum"].data_ptr(),
+                                  P.data_ptr(), y.data_ptr(), _addr(it.get("residual")),
+                                  q.shape[1], y.shape[1], float(it["beta"]), _out_code(y.dtype))
+    return arr
+
+
+def bitlinear_forward_quantized_batch(batch, M, stream=None):
+    _check("bitlinear_forward_quantized_batch", lib().bitlinear_forward_quantized_batch(
+        ctypes.cast(batch, _P), len(batch), M, _stream(stream)))
 
 
 def bitlinear_forward_quantized(q, s_x, rowsum, P, beta, out_dtype=torch.bfloat16, residual=None,

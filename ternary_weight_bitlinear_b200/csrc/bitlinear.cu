@@ -23,6 +23,7 @@ namespace {
 using namespace bl;
 
 constexpr int kQuantThreads = 256;
+constexpr int kSmallBatch = 8;  // parameter-table size of small batches
 
 // ---- device properties and per-kernel launch settings ---------------------
 struct DeviceInfo {
@@ -130,48 +131,114 @@ bl_status check_shape(int64_t M, int64_t K, int64_t N) {
     return BL_OK;
 }
 
-bool decode_eligible(int64_t M, int64_t K) { return M <= kDecMaxTokens && M * K <= kDecMaxQBytes; }
-
 int64_t ws_q_bytes(int64_t M, int64_t K) { return round_up(M * K, 256); }
 int64_t ws_vec_bytes(int64_t M) { return round_up(4 * M, 256); }
+// workspace of one problem: codes | s_x | rowsum
+int64_t ws_problem_bytes(int64_t M, int64_t K) { return ws_q_bytes(M, K) + 2 * ws_vec_bytes(M); }
 
-// ---- decode launches --------------------------------------------------------
-template <int MT, int EPI, bool FUSED>
-bl_status launch_decode_mt(const DecodeArgs& a, int dev, const DeviceInfo& info,
-                           cudaStream_t stream) {
-    const int64_t smem = decode_smem_bytes(MT, a.K, a.chunk);
-    auto fn = decode_kernel<MT, EPI, FUSED>;
-    const int per_sm = prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, kDecThreads,
-                                      smem);
-    if (per_sm < 0) return BL_ERR_CUDA;
-    const int64_t grid = std::min<int64_t>(a.R, (int64_t)info.sms * per_sm);
-    return launch(fn, dim3((unsigned)grid), dim3(kDecThreads), (size_t)smem, stream, a);
+struct WsSlices {
+    int8_t* q;
+    float* s_x;
+    int32_t* rowsum;
+};
+
+WsSlices ws_slices(char* w, int64_t M, int64_t K) {
+    return {reinterpret_cast<int8_t*>(w), reinterpret_cast<float*>(w + ws_q_bytes(M, K)),
+            reinterpret_cast<int32_t*>(w + ws_q_bytes(M, K) + ws_vec_bytes(M))};
 }
 
-template <int EPI, bool FUSED>
-bl_status launch_decode(int mt, const DecodeArgs& a, int dev, const DeviceInfo& info,
-                        cudaStream_t stream) {
+// ---- quantisation launches --------------------------------------------------
+template <int CAP>
+bl_status launch_quant_cap(const QuantProblem* probs, int count, int64_t M, float eps, int dev,
+                           const DeviceInfo& info, cudaStream_t stream) {
+    QuantBatch<CAP> b{};
+    b.count = count;
+    b.M = (int)M;
+    b.eps = eps;
+    int kmax = 16;
+    for (int i = 0; i < count; ++i) {
+        b.p[i] = probs[i];
+        kmax = std::max(kmax, probs[i].K);
+    }
+    auto fn = quant_batch_kernel<kQuantThreads, CAP>;
+    const int64_t smem = 2 * (int64_t)kmax;  // the staged bf16 row
+    if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, kQuantThreads, smem) < 0)
+        return BL_ERR_CUDA;
+    return launch(fn, dim3((unsigned)(count * M)), dim3(kQuantThreads), (size_t)smem, stream, b);
+}
+
+bl_status run_quant(const QuantProblem* probs, int count, int64_t M, float eps, int dev,
+                    const DeviceInfo& info, cudaStream_t stream) {
+    if (count <= kSmallBatch)
+        return launch_quant_cap<kSmallBatch>(probs, count, M, eps, dev, info, stream);
+    return launch_quant_cap<BL_MAX_BATCH>(probs, count, M, eps, dev, info, stream);
+}
+
+// ---- decode launches --------------------------------------------------------
+// One matmul problem on already-quantised codes.
+struct DecodeJob {
+    const int8_t* q;
+    const float* s_x;
+    const int32_t* rowsum;
+    const uint8_t* P;
+    void* y;
+    const uint16_t* residual;
+    int64_t K, N;
+    float beta;
+    int epi;
+};
+
+template <int MT, int CAP>
+bl_status launch_decode_mt(const DecBatch<CAP>& b, int64_t rows, int dev, const DeviceInfo& info,
+                           cudaStream_t stream) {
+    auto fn = decode_batch_kernel<MT, CAP>;
+    if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, kDecThreads, kDecSmemBytes) < 0)
+        return BL_ERR_CUDA;
+    // one CTA per SM: leaves room on every SM for the next kernel's CTAs to
+    // start prefetching (programmatic dependent launch)
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(rows, info.sms));
+    return launch(fn, dim3((unsigned)grid), dim3(kDecThreads), (size_t)kDecSmemBytes, stream, b);
+}
+
+template <int CAP>
+bl_status launch_decode_cap(const DecodeJob* jobs, int count, int mt, int dev,
+                            const DeviceInfo& info, cudaStream_t stream) {
+    DecBatch<CAP> b{};
+    b.count = count;
+    int64_t total = 0, rows = 0;
+    for (int i = 0; i < count; ++i) {
+        DecProblem& p = b.p[i];
+        p.q = jobs[i].q;
+        p.s_x = jobs[i].s_x;
+        p.rowsum = jobs[i].rowsum;
+        p.P = jobs[i].P;
+        p.y = jobs[i].y;
+        p.residual = jobs[i].residual;
+        p.R = jobs[i].N / 4;
+        p.N = jobs[i].N;
+        p.byte0 = total;
+        p.K = (int)jobs[i].K;
+        p.beta = jobs[i].beta;
+        p.epi = jobs[i].epi;
+        total += p.R * p.K;
+        rows += p.R;
+    }
+    b.total = total;
     switch (mt) {
-        case 1: return launch_decode_mt<1, EPI, FUSED>(a, dev, info, stream);
-        case 2: return launch_decode_mt<2, EPI, FUSED>(a, dev, info, stream);
-        case 3: return launch_decode_mt<3, EPI, FUSED>(a, dev, info, stream);
-        case 4: return launch_decode_mt<4, EPI, FUSED>(a, dev, info, stream);
+        case 1: return launch_decode_mt<1, CAP>(b, rows, dev, info, stream);
+        case 2: return launch_decode_mt<2, CAP>(b, rows, dev, info, stream);
+        case 3: return launch_decode_mt<3, CAP>(b, rows, dev, info, stream);
+        case 4: return launch_decode_mt<4, CAP>(b, rows, dev, info, stream);
         default: return BL_ERR_SHAPE;
     }
 }
 
-template <bool FUSED>
-bl_status launch_decode_epi(int epi, int mt, const DecodeArgs& a, int dev, const DeviceInfo& info,
-                            cudaStream_t stream) {
-    switch (epi) {
-        case kEpiF32: return launch_decode<kEpiF32, FUSED>(mt, a, dev, info, stream);
-        case kEpiBF16: return launch_decode<kEpiBF16, FUSED>(mt, a, dev, info, stream);
-        case kEpiI32: return launch_decode<kEpiI32, FUSED>(mt, a, dev, info, stream);
-        default: return BL_ERR_DTYPE;
-    }
+// All jobs share the token count mt (1..4); one launch streams every weight once.
+bl_status run_decode(const DecodeJob* jobs, int count, int mt, int dev, const DeviceInfo& info,
+                     cudaStream_t stream) {
+    if (count <= kSmallBatch) return launch_decode_cap<kSmallBatch>(jobs, count, mt, dev, info, stream);
+    return launch_decode_cap<BL_MAX_BATCH>(jobs, count, mt, dev, info, stream);
 }
-
-int decode_chunk(int64_t K) { return (int)std::min<int64_t>(K, kDecChunkMax); }
 
 // Matmul + epilogue on pre-quantised activations, any M: token groups of up
 // to four rows through the decode kernel.
@@ -179,23 +246,21 @@ bl_status run_quantized(const int8_t* q, const float* s_x, const int32_t* rowsum
                         float beta, int64_t M, int64_t K, int64_t N, void* y, int epi,
                         const uint16_t* residual, int dev, const DeviceInfo& info,
                         cudaStream_t stream) {
-    const int64_t max_mt = std::max<int64_t>(1, std::min<int64_t>(kDecMaxTokens, kDecMaxQBytes / K));
     const size_t ysz = epi == kEpiBF16 ? 2 : 4;
-    for (int64_t m0 = 0; m0 < M; m0 += max_mt) {
-        const int mt = (int)std::min<int64_t>(max_mt, M - m0);
-        DecodeArgs a = {};
-        a.q = q + m0 * K;
-        a.s_x = s_x ? s_x + m0 : nullptr;
-        a.rowsum = rowsum + m0;
-        a.P = P;
-        a.beta = beta;
-        a.K = (int)K;
-        a.chunk = decode_chunk(K);
-        a.R = N / 4;
-        a.N = N;
-        a.y = static_cast<char*>(y) + (size_t)(m0 * N) * ysz;
-        a.residual = residual ? residual + m0 * N : nullptr;
-        bl_status st = launch_decode_epi<false>(epi, mt, a, dev, info, stream);
+    for (int64_t m0 = 0; m0 < M; m0 += kDecMaxTokens) {
+        const int mt = (int)std::min<int64_t>(kDecMaxTokens, M - m0);
+        DecodeJob j;
+        j.q = q + m0 * K;
+        j.s_x = s_x ? s_x + m0 : nullptr;
+        j.rowsum = rowsum + m0;
+        j.P = P;
+        j.y = static_cast<char*>(y) + (size_t)(m0 * N) * ysz;
+        j.residual = residual ? residual + m0 * N : nullptr;
+        j.K = K;
+        j.N = N;
+        j.beta = beta;
+        j.epi = epi;
+        bl_status st = run_decode(&j, 1, mt, dev, info, stream);
         if (st != BL_OK) return st;
     }
     return BL_OK;
@@ -321,17 +386,15 @@ bl_status bitlinear_act_quant(const uint16_t* x, const uint16_t* gain, float eps
     int dev;
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != BL_OK) return st;
-    return launch(act_quant_kernel<kQuantThreads>, dim3((unsigned)M), dim3(kQuantThreads), 0,
-                  static_cast<cudaStream_t>(stream), x, gain, eps, (int)K, q, s_x, rowsum);
+    QuantProblem qp = {x, gain, q, s_x, rowsum, (int)K};
+    return run_quant(&qp, 1, M, eps, dev, info, static_cast<cudaStream_t>(stream));
 }
 
 bl_status bitlinear_forward_workspace_size(int64_t M, int64_t K, int64_t N, size_t* bytes) {
     if (!bytes) return BL_ERR_NULL;
     bl_status st = check_shape(M, K, N);
     if (st != BL_OK) return st;
-    *bytes = (M == 0 || decode_eligible(M, K))
-                 ? 0
-                 : (size_t)(ws_q_bytes(M, K) + 2 * ws_vec_bytes(M));
+    *bytes = M == 0 ? 0 : (size_t)ws_problem_bytes(M, K);
     return BL_OK;
 }
 
@@ -347,39 +410,76 @@ bl_status bitlinear_forward(const uint16_t* x, const uint16_t* gain, float eps, 
     if (!x || !P || !y) return BL_ERR_NULL;
     if (!aligned16(x) || !aligned16(P) || !aligned16(y) || (gain && !aligned16(gain)))
         return BL_ERR_ALIGN;
-    size_t need = 0;
-    bitlinear_forward_workspace_size(M, K, N, &need);
-    if (need > 0) {
-        if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
-        if (!aligned16(workspace)) return BL_ERR_ALIGN;
-    }
+    if (!workspace || workspace_bytes < (size_t)ws_problem_bytes(M, K)) return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGN;
     int dev;
     DeviceInfo info;
     if ((st = current_device(&dev, &info)) != BL_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    if (decode_eligible(M, K)) {
-        DecodeArgs a = {};
-        a.x = x;
-        a.gain = gain;
-        a.eps = eps;
-        a.P = P;
-        a.beta = beta;
-        a.K = (int)K;
-        a.chunk = decode_chunk(K);
-        a.R = N / 4;
-        a.N = N;
-        a.y = y;
-        return launch_decode_epi<true>(epi, (int)M, a, dev, info, s);
+    const WsSlices w = ws_slices(static_cast<char*>(workspace), M, K);
+    QuantProblem qp = {x, gain, w.q, w.s_x, w.rowsum, (int)K};
+    if ((st = run_quant(&qp, 1, M, eps, dev, info, s)) != BL_OK) return st;
+    return run_quantized(w.q, w.s_x, w.rowsum, P, beta, M, K, N, y, epi, nullptr, dev, info, s);
+}
+
+bl_status bitlinear_forward_batch_workspace_size(const bl_problem* probs, int count, int64_t M,
+                                                 size_t* bytes) {
+    if (!bytes || !probs) return BL_ERR_NULL;
+    if (count < 1 || count > BL_MAX_BATCH || M < 0 || M * count > INT32_MAX) return BL_ERR_SHAPE;
+    int64_t total = 0;
+    for (int i = 0; i < count; ++i) {
+        bl_status st = check_shape(M, probs[i].K, probs[i].N);
+        if (st != BL_OK) return st;
+        total += M == 0 ? 0 : ws_problem_bytes(M, probs[i].K);
     }
+    *bytes = (size_t)total;
+    return BL_OK;
+}
+
+bl_status bitlinear_forward_batch(const bl_problem* probs, int count, int64_t M, float eps,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+    size_t need = 0;
+    bl_status st = bitlinear_forward_batch_workspace_size(probs, count, M, &need);
+    if (st != BL_OK) return st;
+    for (int i = 0; i < count; ++i) {
+        const bl_problem& p = probs[i];
+        const int epi = epi_of(p.y_dtype);
+        if (epi < 0 || (p.residual && epi != kEpiBF16)) return BL_ERR_DTYPE;
+        if (M == 0) continue;
+        if (!p.x || !p.P || !p.y) return BL_ERR_NULL;
+        if (!aligned16(p.x) || !aligned16(p.P) || !aligned16(p.y) ||
+            (p.gain && !aligned16(p.gain)) || (p.residual && !aligned16(p.residual)))
+            return BL_ERR_ALIGN;
+    }
+    if (M == 0) return BL_OK;
+    if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGN;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    QuantProblem qp[BL_MAX_BATCH];
+    DecodeJob jobs[BL_MAX_BATCH];
     char* w = static_cast<char*>(workspace);
-    int8_t* q = reinterpret_cast<int8_t*>(w);
-    float* sx = reinterpret_cast<float*>(w + ws_q_bytes(M, K));
-    int32_t* rs = reinterpret_cast<int32_t*>(w + ws_q_bytes(M, K) + ws_vec_bytes(M));
-    if ((st = launch(act_quant_kernel<kQuantThreads>, dim3((unsigned)M), dim3(kQuantThreads), 0, s,
-                     x, gain, eps, (int)K, q, sx, rs)) != BL_OK)
-        return st;
-    return run_quantized(q, sx, rs, P, beta, M, K, N, y, epi, nullptr, dev, info, s);
+    for (int i = 0; i < count; ++i) {
+        const bl_problem& p = probs[i];
+        const WsSlices sl = ws_slices(w, M, p.K);
+        w += ws_problem_bytes(M, p.K);
+        qp[i] = {p.x, p.gain, sl.q, sl.s_x, sl.rowsum, (int)p.K};
+        jobs[i] = {sl.q, sl.s_x, sl.rowsum, p.P, p.y, p.residual, p.K, p.N, p.beta,
+                   epi_of(p.y_dtype)};
+    }
+    if ((st = run_quant(qp, count, M, eps, dev, info, s)) != BL_OK) return st;
+    if (M <= kDecMaxTokens) return run_decode(jobs, count, (int)M, dev, info, s);
+    for (int i = 0; i < count; ++i) {
+        const DecodeJob& j = jobs[i];
+        st = run_quantized(j.q, j.s_x, j.rowsum, j.P, j.beta, M, j.K, j.N, j.y, j.epi, j.residual,
+                           dev, info, s);
+        if (st != BL_OK) return st;
+    }
+    return BL_OK;
 }
 
 bl_status bitlinear_forward_quantized(const int8_t* q, const float* s_x, const int32_t* rowsum,
@@ -399,6 +499,40 @@ bl_status bitlinear_forward_quantized(const int8_t* q, const float* s_x, const i
     if ((st = current_device(&dev, &info)) != BL_OK) return st;
     return run_quantized(q, s_x, rowsum, P, beta, M, K, N, y, epi, residual, dev, info,
                          static_cast<cudaStream_t>(stream));
+}
+
+bl_status bitlinear_forward_quantized_batch(const bl_quantized_problem* probs, int count,
+                                            int64_t M, void* stream) {
+    if (!probs) return BL_ERR_NULL;
+    if (count < 1 || count > BL_MAX_BATCH || M < 0) return BL_ERR_SHAPE;
+    DecodeJob jobs[BL_MAX_BATCH];
+    for (int i = 0; i < count; ++i) {
+        const bl_quantized_problem& p = probs[i];
+        bl_status st = check_shape(M, p.K, p.N);
+        if (st != BL_OK) return st;
+        const int epi = epi_of(p.y_dtype);
+        if (epi < 0 || (p.residual && epi != kEpiBF16)) return BL_ERR_DTYPE;
+        if (M == 0) continue;
+        if (!p.q || !p.s_x || !p.rowsum || !p.P || !p.y) return BL_ERR_NULL;
+        if (!aligned16(p.q) || !aligned16(p.P) || !aligned16(p.y) ||
+            (p.residual && !aligned16(p.residual)))
+            return BL_ERR_ALIGN;
+        jobs[i] = {p.q, p.s_x, p.rowsum, p.P, p.y, p.residual, p.K, p.N, p.beta, epi};
+    }
+    if (M == 0) return BL_OK;
+    int dev;
+    DeviceInfo info;
+    bl_status st;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= kDecMaxTokens) return run_decode(jobs, count, (int)M, dev, info, s);
+    for (int i = 0; i < count; ++i) {
+        const DecodeJob& j = jobs[i];
+        st = run_quantized(j.q, j.s_x, j.rowsum, j.P, j.beta, M, j.K, j.N, j.y, j.epi, j.residual,
+                           dev, info, s);
+        if (st != BL_OK) return st;
+    }
+    return BL_OK;
 }
 
 bl_status bitlinear_accumulate(const int8_t* q, const int32_t* rowsum, const uint8_t* P, int64_t M,

@@ -1,4 +1,5 @@
-// decode.cuh -- memory-bound BitLinear GEMV for 1..4 tokens (decode).
+// decode.cuh -- memory-bound BitLinear GEMV for 1..4 tokens (decode), over a
+// batch of independent BitLinear problems in one launch.
 //
 // Computes acc[m,n] = sum_k q[m,k] t[n,k] straight from the 2-bit packed
 // weights ("Transformers 实战 BitNet 1.58 位量化" walkthrough, section
@@ -6,23 +7,28 @@
 // post_quant_process, y = RN32(RN32(acc * beta) / s_x[m]).
 //
 // Design (B200):
-//  * The packed matrix P[N/4, K] is streamed once.  Each CTA owns a contiguous
-//    range of packed rows; each warp owns every 8th row of that range and runs
-//    its own double-buffered pipeline of bulk copies (TMA engine, L2
-//    evict-first) of row chunks into shared memory, signalled by mbarriers.
-//    Copies for the first chunks are issued before the kernel waits on the
-//    previous grid (programmatic dependent launch), so weight traffic overlaps
-//    the previous kernel's tail and this kernel's own activation quantisation.
-//  * With FUSED, every CTA quantises the (tiny) activation rows itself (RMSNorm
-//    + absmax + int8, identical arithmetic to act_quant_kernel) into shared
-//    memory: one launch per forward and no workspace.
+//  * One launch streams the packed weights of every problem in the batch
+//    exactly once.  The batch's packed rows are laid end to end as one byte
+//    range; every warp of the grid owns an equal share of those bytes (whole
+//    rows), so the load is balanced across all 148 SMs whatever the mix of
+//    shapes.
+//  * Each warp runs its own pipeline of bulk copies (TMA engine, no multicast,
+//    L2 evict-first) of row chunks into shared memory, kDecSlots deep,
+//    signalled by mbarriers.  The first copies are issued before the kernel
+//    waits on the kernel before it (programmatic dependent launch), so weight
+//    traffic overlaps the activation quantisation that precedes it.
 //  * Unpacking never materialises ternary values: bit pair i of a packed byte
 //    is selected in place with the mask 3 << 2i, so each 32-bit word gives four
 //    u8 operands code_i << 2i (code = t+1) for dp4a against four int8 codes.
-//    The shift is removed exactly at the end (>> 2i) and t = code - 1 is folded
-//    in with the row sum of the codes: sum q*t = sum q*code - sum q.
+//    The factor 4^i is shifted out exactly at the end and t = code - 1 is
+//    folded in with the row sum of the codes: sum q*t = sum q*code - sum q.
+//  * After the wait, each CTA stages the int8 codes, scales and row sums of the
+//    problems its rows belong to in shared memory (they are reused by every
+//    row of a problem); batches too large to stage read them from L2.
+//  * Everything another kernel wrote (codes, scales, row sums, residual) is
+//    read with ld.global.cg (L2, coherent), never through the non-coherent L1.
 //  * A warp reduces its 4*MT partial sums with shuffles; lane 4m+i writes
-//    output (m, i*N/4 + r).
+//    output (m, i*N/4 + r) of its problem.
 #pragma once
 
 #include "common.cuh"
@@ -30,38 +36,131 @@
 
 namespace bl {
 
-constexpr int kDecThreads = 256;
+constexpr int kDecThreads = 512;
 constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kDecSlots = 2;          // pipeline depth per warp
-constexpr int kDecChunkMax = 4096;    // bytes per slot
+constexpr int kDecSlots = 8;          // copies in flight per warp (one mbarrier each)
+constexpr int kDecChunk = 4096;       // largest single copy: a row, or a piece of a long row
+constexpr int kDecRing = 10240;       // bytes of each warp's ring of copies
 constexpr int kDecMaxTokens = 4;
-constexpr int kDecMaxQBytes = 65536;  // M*K limit of the shared-memory code buffer
+constexpr int kDecQBudget = 48 * 1024;  // shared-memory bytes for staged codes
+constexpr int kDecMaxStaged = 16;       // problems whose codes one CTA can stage
+// Dynamic shared memory: one 8-byte mbarrier per in-flight copy (padded to 128
+// bytes) | rings | staged codes | staged s_x | staged row sums | code offsets.
+constexpr int kDecBarBytes = (8 * kDecWarps * kDecSlots + 127) / 128 * 128;
+constexpr int kDecSlotBytes = kDecWarps * kDecRing;
+static_assert(kDecChunk <= kDecRing && kDecRing % 128 == 0, "ring size");
+constexpr int kDecMetaBytes = kDecMaxStaged * kDecMaxTokens * 8 + kDecMaxStaged * 4;
+// Per-warp queue of the descriptors of copies in flight (issued, not consumed).
+struct ItemDesc {
+    int p;          // problem
+    int r;          // row
+    int c;          // chunk of the row
+    int bytes;
+    uint32_t at;    // ring offset
+    uint32_t used;  // ring bytes it holds (skipped tail + bytes)
+};
+constexpr int kDecDescBytes = kDecWarps * kDecSlots * (int)sizeof(ItemDesc);
+constexpr int kDecSmemBytes =
+    kDecBarBytes + kDecSlotBytes + kDecQBudget + kDecMetaBytes + kDecDescBytes;
+static_assert(8 * kDecWarps * kDecSlots <= kDecBarBytes, "barriers overlap the slots");
+static_assert(kDecBarBytes % 128 == 0 && kDecChunk % 16 == 0, "copy alignment");
+static_assert(kDecSmemBytes <= 227 * 1024, "shared memory budget");
 
 enum Epilogue { kEpiF32 = 0, kEpiBF16 = 1, kEpiI32 = 2 };
 
-struct DecodeArgs {
-    const uint16_t* x;       // FUSED: bf16 [M,K]
-    const uint16_t* gain;    // FUSED: bf16 [K] or nullptr
-    float eps;
-    const int8_t* q;         // !FUSED: int8 [M,K]
-    const float* s_x;        // !FUSED: [M]
-    const int32_t* rowsum;   // !FUSED: [M]
-    const uint8_t* P;        // [R,K]
-    float beta;
-    int K;
-    int chunk;               // bytes per slot, multiple of 16, <= kDecChunkMax
-    int64_t R;               // N/4
-    int64_t N;
-    void* y;                 // [M,N]
+struct DecProblem {
+    const int8_t* q;           // [M,K] codes
+    const float* s_x;          // [M] (unused by kEpiI32)
+    const int32_t* rowsum;     // [M]
+    const uint8_t* P;          // [R,K]
+    void* y;                   // [M,N]
     const uint16_t* residual;  // bf16 [M,N] or nullptr (kEpiBF16 only)
+    int64_t R;                 // N/4
+    int64_t N;
+    int64_t byte0;             // sum of R*K over the problems before this one
+    int K;
+    float beta;
+    int epi;
+};
+
+template <int CAP>
+struct DecBatch {
+    int count;
+    int64_t total;             // sum of R*K over the batch
+    DecProblem p[CAP];
 };
 
 __host__ __device__ constexpr int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
-// Dynamic shared memory: codes | barriers (128 B) | slots.
-__host__ __device__ inline int64_t decode_q_bytes(int mt, int K) { return round_up((int64_t)mt * K, 128); }
-__host__ __device__ inline int64_t decode_smem_bytes(int mt, int K, int chunk) {
-    return decode_q_bytes(mt, K) + 128 + (int64_t)kDecWarps * kDecSlots * chunk;
+// Last problem whose first byte is at or before `pos`.
+template <int CAP>
+__device__ __forceinline__ int problem_at(const DecBatch<CAP>& b, int64_t pos) {
+    int lo_p = 0, hi_p = b.count - 1;
+    while (lo_p < hi_p) {
+        const int mid = (lo_p + hi_p + 1) >> 1;
+        if (b.p[mid].byte0 <= pos) lo_p = mid; else hi_p = mid - 1;
+    }
+    return lo_p;
+}
+
+// A warp's walk over the (problem, row, chunk) items whose rows start in its
+// byte range [lo, hi), with the current problem's constants kept in registers.
+template <int CAP>
+struct Walker {
+    int p;      // current problem; b.count once the walk is over
+    int r;      // row in p
+    int r_end;  // first row of p outside the range
+    int c;      // chunk of the row
+    int K;
+    const uint8_t* P;
+
+    __device__ __forceinline__ void enter(const DecBatch<CAP>& b, int np, int64_t r0, int64_t hi) {
+        p = np;
+        c = 0;
+        if (p >= b.count) return;
+        const DecProblem& pr = b.p[p];
+        K = pr.K;
+        P = pr.P;
+        const int64_t lim = hi - pr.byte0;  // rows with first byte < hi
+        r_end = (int)(lim <= 0 ? 0 : min((lim + K - 1) / K, pr.R));
+        r = (int)min(r0, pr.R);
+    }
+    __device__ __forceinline__ void settle(const DecBatch<CAP>& b, int64_t hi) {
+        while (p < b.count && r >= r_end) {
+            if (r_end < b.p[p].R) { p = b.count; return; }  // the range ends inside p
+            enter(b, p + 1, 0, hi);
+        }
+    }
+    __device__ __forceinline__ void start(const DecBatch<CAP>& b, int64_t lo, int64_t hi) {
+        const int pp = problem_at(b, lo);
+        const DecProblem& pr = b.p[pp];
+        enter(b, pp, (lo - pr.byte0 + pr.K - 1) / pr.K, hi);
+        settle(b, hi);
+    }
+    __device__ __forceinline__ bool valid(const DecBatch<CAP>& b) const { return p < b.count; }
+    __device__ __forceinline__ int bytes() const { return min(kDecChunk, K - c * kDecChunk); }
+    __device__ __forceinline__ bool last_chunk() const { return (c + 1) * kDecChunk >= K; }
+    __device__ __forceinline__ const uint8_t* src() const {
+        return P + (int64_t)r * K + c * kDecChunk;
+    }
+    __device__ __forceinline__ void advance(const DecBatch<CAP>& b, int64_t hi) {
+        if (!last_chunk()) { ++c; return; }
+        c = 0;
+        ++r;
+        settle(b, hi);
+    }
+};
+
+// Placement of the next copy in a warp's byte ring: at `off`, or at the
+// ring's start when it would run past the end; the skipped tail (possibly 0
+// bytes) counts as used until the copy is consumed.
+struct RingSpot {
+    uint32_t at;    // offset of the copy
+    uint32_t used;  // skipped tail + copy bytes
+};
+__device__ __forceinline__ RingSpot ring_spot(uint32_t off, int bytes) {
+    const bool wrap = off + (uint32_t)bytes > (uint32_t)kDecRing;
+    return {wrap ? 0u : off, (wrap ? (uint32_t)kDecRing - off : 0u) + (uint32_t)bytes};
 }
 
 // acc[i] += sum over the 16 bytes of (bit pair i of w, left in place) * q
@@ -77,46 +176,62 @@ __device__ __forceinline__ void dot16(const uint4 w4, const uint4 q4, int (&acc)
     }
 }
 
-template <int EPI>
-__device__ __forceinline__ void store_output(const DecodeArgs& a, int64_t idx, int acc,
-                                             float s_x) {
-    if (EPI == kEpiI32) {
-        static_cast<int32_t*>(a.y)[idx] = acc;
+__device__ __forceinline__ void store_output(const DecProblem& pr, int64_t idx, int acc, float s_x) {
+    if (pr.epi == kEpiI32) {
+        static_cast<int32_t*>(pr.y)[idx] = acc;
+        return;
+    }
+    const float y = __fdiv_rn(__fmul_rn(__int2float_rn(acc), pr.beta), s_x);
+    if (pr.epi == kEpiF32) {
+        static_cast<float*>(pr.y)[idx] = y;
     } else {
-        const float y = __fdiv_rn(__fmul_rn(__int2float_rn(acc), a.beta), s_x);
-        if (EPI == kEpiF32) {
-            static_cast<float*>(a.y)[idx] = y;
-        } else {
-            uint16_t b = float_to_bf16_bits(y);
-            if (a.residual)
-                b = float_to_bf16_bits(__fadd_rn(bf16_bits_to_float(a.residual[idx]),
-                                                 bf16_bits_to_float(b)));
-            static_cast<uint16_t*>(a.y)[idx] = b;
-        }
+        uint16_t b = float_to_bf16_bits(y);
+        if (pr.residual)
+            b = float_to_bf16_bits(
+                __fadd_rn(bf16_bits_to_float(__ldcg(pr.residual + idx)), bf16_bits_to_float(b)));
+        static_cast<uint16_t*>(pr.y)[idx] = b;
     }
 }
 
-template <int MT, int EPI, bool FUSED>
-__global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeArgs a) {
+// Sum 4 per-lane partials over the warp (reduce-scatter: 6 shuffles).  On
+// return lane 8*i holds the total of a[i] (lanes 0, 8, 16, 24).
+__device__ __forceinline__ int warp_reduce4(const int (&a)[4], int lane) {
+    const bool hi16 = lane & 16, hi8 = lane & 8;
+    int k0 = hi16 ? a[2] : a[0], k1 = hi16 ? a[3] : a[1];
+    const int s0 = hi16 ? a[0] : a[2], s1 = hi16 ? a[1] : a[3];
+    k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+    k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+    int k = hi8 ? k1 : k0;
+    k += __shfl_xor_sync(0xffffffffu, hi8 ? k0 : k1, 8);
+    k += __shfl_xor_sync(0xffffffffu, k, 4);
+    k += __shfl_xor_sync(0xffffffffu, k, 2);
+    k += __shfl_xor_sync(0xffffffffu, k, 1);
+    return k;
+}
+
+template <int MT, int CAP>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
+    const __grid_constant__ DecBatch<CAP> b) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ QuantScratch<kDecThreads> sc;
-    __shared__ float s_sx[MT];
-    __shared__ int s_rs[MT];
-
-    const int K = a.K;
-    const int chunk = a.chunk;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    uint8_t* rings = smem + kDecBarBytes;
+    int8_t* qs = reinterpret_cast<int8_t*>(smem + kDecBarBytes + kDecSlotBytes);
+    float* sxs = reinterpret_cast<float*>(smem + kDecBarBytes + kDecSlotBytes + kDecQBudget);
+    int* rss = reinterpret_cast<int*>(sxs + kDecMaxStaged * kDecMaxTokens);
+    int* qoff = rss + kDecMaxStaged * kDecMaxTokens;
+    ItemDesc* descs = reinterpret_cast<ItemDesc*>(
+        smem + kDecBarBytes + kDecSlotBytes + kDecQBudget + kDecMetaBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int8_t* q_s = reinterpret_cast<int8_t*>(smem);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + decode_q_bytes(MT, K));
-    uint8_t* slots = smem + decode_q_bytes(MT, K) + 128;
+    uint8_t* ring = rings + (size_t)warp * kDecRing;
+    ItemDesc* my_descs = descs + warp * kDecSlots;
+    const uint32_t bar0 = smem_addr(&bars[warp * kDecSlots]);  // this warp's barriers
 
-    const int64_t R = a.R;
-    const int64_t r_begin = (R * blockIdx.x) / gridDim.x;
-    const int64_t r_end = (R * (blockIdx.x + 1)) / gridDim.x;
-    const int nck = (K + chunk - 1) / chunk;
-    const int64_t cta_rows = r_end - r_begin;
-    const int64_t my_rows = cta_rows > warp ? (cta_rows - warp + kDecWarps - 1) / kDecWarps : 0;
-    const int64_t n_items = my_rows * nck;  // (row, chunk) pairs of this warp
+    // this warp's (and this CTA's) share of the batch's packed bytes
+    const int64_t W = (int64_t)gridDim.x * kDecWarps;
+    const int64_t gw = (int64_t)blockIdx.x * kDecWarps + warp;
+    const int64_t lo = gw * b.total / W, hi = (gw + 1) * b.total / W;
+    const int64_t clo = (int64_t)blockIdx.x * kDecWarps * b.total / W;
+    const int64_t chi = ((int64_t)blockIdx.x + 1) * kDecWarps * b.total / W;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDecWarps * kDecSlots; ++i) mbar_init(smem_addr(&bars[i]), 1);
@@ -124,102 +239,146 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeArgs a)
     }
     __syncthreads();
 
+    // The only walk over this warp's items is the issuing one; each issued
+    // copy leaves its descriptor in the warp's queue for the consumer.
     const uint64_t policy = policy_evict_first();
-    auto issue = [&](int64_t item) {  // lane 0 only
-        const int64_t r = r_begin + warp + (int64_t)kDecWarps * (item / nck);
-        const int k0 = (int)(item % nck) * chunk;
-        const int bytes = min(chunk, K - k0);
-        const int slot = (int)(item % kDecSlots);
-        const uint32_t bar = smem_addr(&bars[warp * kDecSlots + slot]);
-        mbar_arrive_expect_tx(bar, (uint32_t)bytes);
-        bulk_g2s_stream(smem_addr(slots + (size_t)(warp * kDecSlots + slot) * chunk),
-                        a.P + r * K + k0, (uint32_t)bytes, bar, policy);
+    Walker<CAP> iw;
+    iw.start(b, lo, hi);
+    uint32_t issued = 0, done = 0;                      // items
+    uint32_t ioff = 0, ring_free = kDecRing;            // ring bookkeeping (bytes)
+    auto refill = [&]() {
+        while (issued - done < (uint32_t)kDecSlots && iw.valid(b)) {
+            const int bytes = iw.bytes();
+            const RingSpot spot = ring_spot(ioff, bytes);
+            if (spot.used > ring_free) break;
+            const uint32_t bar = bar0 + 8u * (issued % kDecSlots);
+            if (lane == 0) {
+                my_descs[issued % kDecSlots] = ItemDesc{iw.p, iw.r, iw.c, bytes, spot.at, spot.used};
+                fence_proxy_async_smem();  // this warp's earlier reads of the ring come first
+                mbar_arrive_expect_tx(bar, (uint32_t)bytes);
+                bulk_g2s_stream(smem_addr(ring + spot.at), iw.src(), (uint32_t)bytes, bar, policy);
+            }
+            ring_free -= spot.used;
+            ioff = spot.at + (uint32_t)bytes;
+            ++issued;
+            iw.advance(b, hi);
+        }
+        __syncwarp();  // descriptors written by lane 0 are visible to the warp
     };
-    if (lane == 0)
-        for (int64_t it = 0; it < n_items && it < kDecSlots; ++it) issue(it);
+    refill();
 
-    // Everything above touches only the (constant) weights.
+    // Everything above touches only the (constant) weights.  Dependents are
+    // released only after this grid's own inputs are complete, so no kernel
+    // runs more than one launch ahead of the data it reads.
     pdl_wait();
     pdl_launch_dependents();
 
-    if (FUSED) {
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            float s;
-            int rs;
-            quantize_row<kDecThreads>(a.x + (int64_t)m * K, a.gain, a.eps, K, q_s + m * K, sc, s,
-                                      rs);
-            if (threadIdx.x == 0) { s_sx[m] = s; s_rs[m] = rs; }
-        }
-    } else {
-        const int nv = MT * K / 16;
-        for (int v = threadIdx.x; v < nv; v += kDecThreads)
-            reinterpret_cast<uint4*>(q_s)[v] = __ldg(reinterpret_cast<const uint4*>(a.q) + v);
-        if (threadIdx.x < MT) {
-            s_sx[threadIdx.x] = a.s_x ? a.s_x[threadIdx.x] : 1.0f;  // unused by kEpiI32
-            s_rs[threadIdx.x] = a.rowsum[threadIdx.x];
+    // Stage the codes, scales and row sums of the problems this CTA touches
+    // (rows starting in [clo, chi)): they are reused by every row of a problem.
+    Walker<CAP> cta;
+    cta.start(b, clo, chi);
+    const int pa = cta.p;
+    const int pb = chi > 0 ? problem_at(b, chi - 1) : -1;
+    int64_t need = 0;
+    for (int p = pa; p <= pb; ++p) need += (int64_t)MT * b.p[p].K;
+    const bool staged = cta.valid(b) && pb - pa + 1 <= kDecMaxStaged && need <= kDecQBudget;
+    if (staged) {
+        int off = 0;
+        for (int p = pa; p <= pb; ++p) {
+            const DecProblem& pr = b.p[p];
+            const int nv = MT * pr.K / 16;
+            const uint4* src = reinterpret_cast<const uint4*>(pr.q);
+            uint4* dst = reinterpret_cast<uint4*>(qs + off);
+            for (int v = threadIdx.x; v < nv; v += kDecThreads) dst[v] = __ldcg(src + v);
+            if (threadIdx.x < MT) {
+                sxs[(p - pa) * kDecMaxTokens + threadIdx.x] =
+                    pr.epi == kEpiI32 ? 1.0f : __ldcg(pr.s_x + threadIdx.x);
+                rss[(p - pa) * kDecMaxTokens + threadIdx.x] = __ldcg(pr.rowsum + threadIdx.x);
+            }
+            if (threadIdx.x == 0) qoff[p - pa] = off;
+            off += MT * pr.K;
         }
     }
     __syncthreads();
 
-    int64_t it = 0;
     bool ok = true;
-    for (int64_t row = warp; row < cta_rows; row += kDecWarps) {
-        int acc[MT][4];
+    int acc[MT][4];
+    int cur_p = -1, K = 0;
+    const int8_t* qbase = nullptr;
+    float sx[MT];
+    int rsum[MT];
+    while (done < issued) {  // refill() keeps the queue non-empty until the walk ends
+        const ItemDesc d = my_descs[done % kDecSlots];
+        if (d.p != cur_p) {  // entering a problem: cache its activation data
+            cur_p = d.p;
+            const DecProblem& pr = b.p[cur_p];
+            K = pr.K;
+            if (staged) {
+                qbase = qs + qoff[cur_p - pa];
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
+                for (int m = 0; m < MT; ++m) {
+                    sx[m] = sxs[(cur_p - pa) * kDecMaxTokens + m];
+                    rsum[m] = rss[(cur_p - pa) * kDecMaxTokens + m];
+                }
+            } else {
+                qbase = pr.q;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) acc[m][i] = 0;
-
-        for (int c = 0; c < nck; ++c, ++it) {
-            const int slot = (int)(it % kDecSlots);
-            const uint32_t parity = (uint32_t)((it / kDecSlots) & 1);
-            const bool got = mbar_wait(smem_addr(&bars[warp * kDecSlots + slot]), parity);
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-            const int k0 = c * chunk;
-            const int nvec = min(chunk, K - k0) >> 4;
-            const uint4* wp =
-                reinterpret_cast<const uint4*>(slots + (size_t)(warp * kDecSlots + slot) * chunk);
+                for (int m = 0; m < MT; ++m) {
+                    sx[m] = pr.epi == kEpiI32 ? 1.0f : __ldcg(pr.s_x + m);
+                    rsum[m] = __ldcg(pr.rowsum + m);
+                }
+            }
+        }
+        if (d.c == 0) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[m][i] = 0;
+        }
+        const bool got = mbar_wait(bar0 + 8u * (done % kDecSlots), (done / kDecSlots) & 1u);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        const uint4* wp = reinterpret_cast<const uint4*>(ring + d.at);
+        const int nvec = d.bytes >> 4;
+        const int8_t* qrow = qbase + d.c * kDecChunk;
+        if (staged) {
+#pragma unroll 4
             for (int v = lane; v < nvec; v += 32) {
                 const uint4 w4 = wp[v];
 #pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    const uint4 q4 = *reinterpret_cast<const uint4*>(q_s + m * K + k0 + 16 * v);
-                    dot16(w4, q4, acc[m]);
-                }
+                for (int m = 0; m < MT; ++m)
+                    dot16(w4, reinterpret_cast<const uint4*>(qrow + m * K)[v], acc[m]);
             }
-            __syncwarp();
-            if (lane == 0 && it + kDecSlots < n_items) {
-                fence_proxy_async_smem();  // our reads of this slot precede its refill
-                issue(it + kDecSlots);
+        } else {
+            for (int v = lane; v < nvec; v += 32) {
+                const uint4 w4 = wp[v];
+#pragma unroll
+                for (int m = 0; m < MT; ++m)
+                    dot16(w4, __ldcg(reinterpret_cast<const uint4*>(qrow + (int64_t)m * K) + v),
+                          acc[m]);
             }
         }
-        if (!ok) break;
-
+        __syncwarp();
+        ring_free += d.used;
+        ++done;
+        refill();
+        if ((d.c + 1) * kDecChunk >= K) {  // last chunk of the row: reduce and store
+            const DecProblem& pr = b.p[cur_p];
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    acc[m][i] += __shfl_xor_sync(0xffffffffu, acc[m][i], o);
-
-        const int64_t r = r_begin + row;
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                if (lane == 4 * m + i) {
-                    const int exact = (acc[m][i] >> (2 * i)) - s_rs[m];
-                    store_output<EPI>(a, (int64_t)m * a.N + (int64_t)i * R + r, exact, s_sx[m]);
+            for (int m = 0; m < MT; ++m) {
+                const int tot = warp_reduce4(acc[m], lane);
+                if ((lane & 7) == 0) {
+                    const int i = lane >> 3;
+                    store_output(pr, (int64_t)m * pr.N + (int64_t)i * pr.R + d.r,
+                                 (tot >> (2 * i)) - rsum[m], sx[m]);
                 }
+            }
+        }
     }
 
     if (!ok && lane == 0) {
-        // Drain copies still in flight into this warp's slots before exiting.
-        for (int64_t j = it; j < n_items && j < it + kDecSlots; ++j)
-            mbar_wait(smem_addr(&bars[warp * kDecSlots + (int)(j % kDecSlots)]),
-                      (uint32_t)((j / kDecSlots) & 1));
+        // Drain the copies still in flight into this warp's ring before exiting.
+        for (uint32_t j = done; j < issued; ++j)
+            mbar_wait(bar0 + 8u * (j % kDecSlots), (j / kDecSlots) & 1u);
     }
 }
 

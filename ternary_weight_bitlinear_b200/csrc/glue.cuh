@@ -27,8 +27,8 @@ __global__ void __launch_bounds__(kGlueThreads) relu2_mul_kernel(const uint16_t*
     const int64_t base = ((int64_t)blockIdx.x * kGlueThreads + threadIdx.x) * 8;
     if (base >= n) return;
     if (base + 8 <= n) {
-        const uint4 ua = *reinterpret_cast<const uint4*>(a + base);
-        const uint4 ub = *reinterpret_cast<const uint4*>(b + base);
+        const uint4 ua = __ldcg(reinterpret_cast<const uint4*>(a + base));
+        const uint4 ub = __ldcg(reinterpret_cast<const uint4*>(b + base));
         const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
         const uint32_t wb[4] = {ub.x, ub.y, ub.z, ub.w};
         uint32_t o[4];
@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(kGlueThreads) relu2_mul_kernel(const uint16_t*
                    ((uint32_t)relu2_mul_one(wa[j] >> 16, wb[j] >> 16) << 16);
         *reinterpret_cast<uint4*>(z + base) = make_uint4(o[0], o[1], o[2], o[3]);
     } else {
-        for (int64_t i = base; i < n; ++i) z[i] = relu2_mul_one(a[i], b[i]);
+        for (int64_t i = base; i < n; ++i) z[i] = relu2_mul_one(__ldcg(a + i), __ldcg(b + i));
     }
 }
 

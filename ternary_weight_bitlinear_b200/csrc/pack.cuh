@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(kPackThreads) absmean_partial_kernel(
     const float4* wv = reinterpret_cast<const float4*>(W);
     const int64_t stride = (int64_t)gridDim.x * kPackThreads;
     for (int64_t v = (int64_t)blockIdx.x * kPackThreads + threadIdx.x; v < nvec; v += stride) {
-        const float4 f = __ldg(wv + v);
+        const float4 f = __ldcg(wv + v);
         dd_add(hi, lo, fabs((double)f.x));
         dd_add(hi, lo, fabs((double)f.y));
         dd_add(hi, lo, fabs((double)f.z));
@@ -63,8 +63,8 @@ __global__ void absmean_finalize_kernel(int64_t n, int parts, PackWorkspace* __r
                                         float* __restrict__ beta_out) {
     pdl_wait();
     if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    double h = ws->part_hi[0], l = ws->part_lo[0];
-    for (int p = 1; p < parts; ++p) dd_merge(h, l, ws->part_hi[p], ws->part_lo[p]);
+    double h = __ldcg(&ws->part_hi[0]), l = __ldcg(&ws->part_lo[0]);
+    for (int p = 1; p < parts; ++p) dd_merge(h, l, __ldcg(&ws->part_hi[p]), __ldcg(&ws->part_lo[p]));
     const double sum = __dadd_rn(h, l);
     const double mean = __ddiv_rn(sum, (double)n);
     const float beta = fmaxf(__double2float_rn(mean), kScaleFloor);
@@ -87,14 +87,14 @@ __global__ void __launch_bounds__(kPackThreads) ternarize_pack_kernel(
     const int64_t idx = (int64_t)blockIdx.x * kPackThreads + threadIdx.x;
     if (idx >= R * cols16) return;
     const int64_t r = idx / cols16, c = idx - r * cols16;
-    const float s_w = ws->s_w;
+    const float s_w = __ldcg(&ws->s_w);
     uint32_t out[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const float4* src = reinterpret_cast<const float4*>(W + (i * R + r) * K + c * 16);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-            const float4 f = __ldg(src + v);
+            const float4 f = __ldcg(src + v);
             const float e[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j)  // column c*16 + 4v + j -> byte 4v + j
@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_ternary_kernel(
     uint32_t out[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(t + (i * R + r) * K) + c);
+        const uint4 u = __ldcg(reinterpret_cast<const uint4*>(t + (i * R + r) * K) + c);
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kPackThreads) unpack_kernel(
     const int64_t idx = (int64_t)blockIdx.x * kPackThreads + threadIdx.x;
     if (idx >= R * cols16) return;
     const int64_t r = idx / cols16, c = idx - r * cols16;
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(P + r * K) + c);
+    const uint4 u = __ldcg(reinterpret_cast<const uint4*>(P + r * K) + c);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {

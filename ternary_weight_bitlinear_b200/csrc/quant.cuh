@@ -8,7 +8,7 @@
 // reduction order), so r = RN32(1/sqrt(SS/K + eps)) is reproducible bit for bit.
 //
 // One CTA works on one token row; all loads are 16-byte vectors (8 bf16).  The
-// row is re-read from L1 in each pass instead of being staged.
+// row is read from global memory once and staged in shared memory.
 #pragma once
 
 #include "common.cuh"
@@ -95,14 +95,15 @@ __device__ __forceinline__ float norm_elem(float x, float r, float g) {
     return __fmul_rn(__fmul_rn(x, r), g);
 }
 
-// Quantise one token row.  x: K bf16 (global, 16-byte aligned); gain: K bf16
-// or nullptr (no norm); q: K int8 destination (global or shared, 8-byte
-// aligned).  Every thread of the CTA must call it; s_out and rowsum_out are
-// valid in every thread on return.
+// Quantise one token row.  x: K bf16 (global, 16-byte aligned), read once
+// with ld.global.cg (it may have just been written by the previous kernel) and
+// staged in xs (shared, K/8 vectors); gain: K bf16 or nullptr (no norm); q: K
+// int8 destination (global, 8-byte aligned).  Every thread of the CTA must
+// call it; s_out and rowsum_out are valid in every thread on return.
 template <int NT>
 __device__ void quantize_row(const uint16_t* __restrict__ x, const uint16_t* __restrict__ gain,
-                             float eps, int K, int8_t* __restrict__ q, QuantScratch<NT>& sc,
-                             float& s_out, int& rowsum_out) {
+                             float eps, int K, int8_t* __restrict__ q, uint4* __restrict__ xs,
+                             QuantScratch<NT>& sc, float& s_out, int& rowsum_out) {
     const int nvec = K >> 3;
     const uint4* xv = reinterpret_cast<const uint4*>(x);
     const uint4* gv = reinterpret_cast<const uint4*>(gain);
@@ -113,8 +114,10 @@ __device__ void quantize_row(const uint16_t* __restrict__ x, const uint16_t* __r
     if (norm) {
         double hi = 0.0, lo = 0.0;
         for (int v = threadIdx.x; v < nvec; v += NT) {
+            const uint4 u = __ldcg(xv + v);
+            xs[v] = u;
             float f[8];
-            unpack8_bf16(__ldg(xv + v), f);
+            unpack8_bf16(u, f);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const double d = (double)f[j];
@@ -129,15 +132,17 @@ __device__ void quantize_row(const uint16_t* __restrict__ x, const uint16_t* __r
         r = __double2float_rn(rd);
         for (int v = threadIdx.x; v < nvec; v += NT) {
             float f[8], g[8];
-            unpack8_bf16(__ldg(xv + v), f);
+            unpack8_bf16(xs[v], f);
             unpack8_bf16(__ldg(gv + v), g);
 #pragma unroll
             for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(norm_elem(f[j], r, g[j])));
         }
     } else {
         for (int v = threadIdx.x; v < nvec; v += NT) {
+            const uint4 u = __ldcg(xv + v);
+            xs[v] = u;
             float f[8];
-            unpack8_bf16(__ldg(xv + v), f);
+            unpack8_bf16(u, f);
 #pragma unroll
             for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(f[j]));
         }
@@ -148,7 +153,7 @@ __device__ void quantize_row(const uint16_t* __restrict__ x, const uint16_t* __r
     int rs = 0;
     for (int v = threadIdx.x; v < nvec; v += NT) {
         float f[8], g[8];
-        unpack8_bf16(__ldg(xv + v), f);
+        unpack8_bf16(xs[v], f);
         if (norm) {
             unpack8_bf16(__ldg(gv + v), g);
 #pragma unroll
@@ -168,24 +173,42 @@ __device__ void quantize_row(const uint16_t* __restrict__ x, const uint16_t* __r
     s_out = s;
 }
 
-// bitlinear_act_quant: one CTA per token row.
-template <int NT>
-__global__ void __launch_bounds__(NT) act_quant_kernel(const uint16_t* __restrict__ x,
-                                                       const uint16_t* __restrict__ gain,
-                                                       float eps, int K,
-                                                       int8_t* __restrict__ q,
-                                                       float* __restrict__ s_x,
-                                                       int32_t* __restrict__ rowsum) {
+// ---- one CTA per (problem, token row) of a batch ----------------------------
+struct QuantProblem {
+    const uint16_t* x;     // bf16 [M,K]
+    const uint16_t* gain;  // bf16 [K] or nullptr
+    int8_t* q;             // [M,K]
+    float* s_x;            // [M]
+    int32_t* rowsum;       // [M] or nullptr
+    int K;
+};
+
+template <int CAP>
+struct QuantBatch {
+    int count;
+    int M;
+    float eps;
+    QuantProblem p[CAP];
+};
+
+// Dynamic shared memory: 2 * max K bytes (the staged row).
+template <int NT, int CAP>
+__global__ void __launch_bounds__(NT) quant_batch_kernel(const __grid_constant__ QuantBatch<CAP> b) {
+    extern __shared__ __align__(16) uint4 xs[];
     __shared__ QuantScratch<NT> sc;
-    pdl_wait();
+    // The kernel after this one only prefetches constant weights before it
+    // waits for this grid, so it may launch right away.
     pdl_launch_dependents();
-    const int64_t m = blockIdx.x;
+    pdl_wait();
+    const int p = blockIdx.x / b.M, m = blockIdx.x % b.M;
+    const QuantProblem& pr = b.p[p];
     float s;
     int rs;
-    quantize_row<NT>(x + m * K, gain, eps, K, q + m * K, sc, s, rs);
+    quantize_row<NT>(pr.x + (int64_t)m * pr.K, pr.gain, b.eps, pr.K, pr.q + (int64_t)m * pr.K, xs,
+                     sc, s, rs);
     if (threadIdx.x == 0) {
-        s_x[m] = s;
-        if (rowsum) rowsum[m] = rs;
+        pr.s_x[m] = s;
+        if (pr.rowsum) pr.rowsum[m] = rs;
     }
 }
 

@@ -44,8 +44,8 @@ def test_abi_version_and_status_strings(L):
 
 
 def test_workspace_sizes(L):
-    assert B.bitlinear_forward_workspace_size(1, 2560, 6912) == 0
-    assert B.bitlinear_forward_workspace_size(4, 6912, 2560) == 0
+    assert B.bitlinear_forward_workspace_size(1, 2560, 6912) >= 2560 + 8
+    assert B.bitlinear_forward_workspace_size(4, 6912, 2560) >= 4 * 6912 + 32
     assert B.bitlinear_forward_workspace_size(0, 2560, 2560) == 0
     big = B.bitlinear_forward_workspace_size(4096, 2560, 6912)
     assert big >= 4096 * 2560 + 2 * 4096 * 4
@@ -54,7 +54,7 @@ def test_workspace_sizes(L):
         B.bitlinear_forward_workspace_size(1, 2561, 16)
 
 
-def _fwd(L, x=P16, gain=NULL, P=P16, M=1, K=256, N=128, y=P16, dt=0, ws=NULL, wsb=0):
+def _fwd(L, x=P16, gain=NULL, P=P16, M=1, K=256, N=128, y=P16, dt=0, ws=P16, wsb=1 << 30):
     return L.bitlinear_forward(x, gain, 1e-5, P, 1.0, M, K, N, y, dt, ws, wsb, NULL)
 
 
@@ -70,8 +70,9 @@ def test_forward_argument_checks(L):
     assert _fwd(L, y=NULL) == 1
     assert _fwd(L, x=P17) == 3
     assert _fwd(L, gain=P17) == 3
-    assert _fwd(L, M=64, K=2560) == 5   # needs a workspace
+    assert _fwd(L, M=64, K=2560, ws=NULL) == 5   # needs a workspace
     assert _fwd(L, M=64, K=2560, ws=P16, wsb=16) == 5
+    assert _fwd(L, ws=P17) == 3
 
 
 def test_other_entry_points_check_arguments(L):
@@ -95,6 +96,31 @@ def test_no_device_is_reported_not_faked(L):
     assert _fwd(L) == 8
     assert L.bitlinear_act_quant(P16, NULL, 1e-5, 2, 64, P16, P16, P16, NULL) == 8
     assert L.bitlinear_device_status(NULL) == 8
+
+
+def _batch(n, K=256, N=128, x=P16, dt=0, residual=None):
+    arr = (B.bitlinear.Problem * n)()
+    for i in range(n):
+        arr[i] = B.bitlinear.Problem(x.value, None, P16.value, P16.value,
+                                     residual.value if residual else None, K, N, 1.0, dt)
+    return arr
+
+
+def test_batch_argument_checks(L):
+    sz = ctypes.c_size_t()
+    arr = _batch(7)
+    assert L.bitlinear_forward_batch_workspace_size(arr, 7, 1, ctypes.byref(sz)) == 0
+    assert sz.value == 7 * B.bitlinear_forward_workspace_size(1, 256, 128)
+    assert L.bitlinear_forward_batch_workspace_size(arr, 0, 1, ctypes.byref(sz)) == 2
+    big = _batch(257)
+    assert L.bitlinear_forward_batch_workspace_size(big, 257, 1, ctypes.byref(sz)) == 2
+    assert L.bitlinear_forward_batch(_batch(3, K=250), 3, 1, 1e-5, P16, 1 << 30, NULL) == 2
+    assert L.bitlinear_forward_batch(_batch(3, dt=9), 3, 1, 1e-5, P16, 1 << 30, NULL) == 4
+    assert L.bitlinear_forward_batch(_batch(3, dt=1, residual=P16), 3, 1, 1e-5, P16, 1 << 30,
+                                     NULL) == 4
+    assert L.bitlinear_forward_batch(_batch(3, x=P17), 3, 1, 1e-5, P16, 1 << 30, NULL) == 3
+    assert L.bitlinear_forward_batch(arr, 7, 1, 1e-5, NULL, 0, NULL) == 5
+    assert L.bitlinear_forward_batch(arr, 7, 0, 1e-5, NULL, 0, NULL) == 0  # M = 0: no-op
 
 
 def test_binding_rejects_cpu_tensors():

@@ -247,3 +247,101 @@ def test_ragged_and_extreme_shapes(M, K, N):
     for norm in (False, True):
         c = dict(x=x, gain=g, norm=norm, out="f32")
         run_forward(c, P_d, beta, P_o, beta_o, "M=%d K=%d N=%d norm=%s" % (M, K, N, norm))
+
+
+# ---------------------------------------------------------------------------
+# batched forwards (independent problems in one call)
+# ---------------------------------------------------------------------------
+def _batch_case(specs, M, seed):
+    """specs: list of (K, N, norm, out dtype, residual) -> (items, oracle outputs)."""
+    items, refs = [], []
+    for i, (K, N, norm, dt, res) in enumerate(specs):
+        x = WL.activations(M, K, seed=seed + i, outlier_frac=0.001)
+        g = WL.gain(K, seed=seed + 100 + i) if norm else None
+        P_d, beta, P_o, beta_o = both_pack(WL.master_weights(N, K, seed=seed + 200 + i))
+        y_o = O.forward(x, P_o, beta_o, gain=g, eps=WL.RMS_EPS, norm=norm)["y"]
+        it = dict(x=bf16_dev(x), P=P_d, beta=beta, y=torch.empty((M, N), dtype=dt, device="cuda"))
+        if norm:
+            it["gain"] = bf16_dev(g)
+        if res:
+            r = WL.activations(M, N, seed=seed + 300 + i)
+            it["residual"] = bf16_dev(r)
+            refs.append(("bf16", O.residual_add(r, O.f32_to_bf16(y_o))))
+        elif dt == torch.float32:
+            refs.append(("f32", y_o))
+        else:
+            refs.append(("bf16", O.f32_to_bf16(y_o)))
+        items.append(it)
+    return items, refs
+
+
+def _check_batch(items, refs, what):
+    for i, (it, (kind, ref)) in enumerate(zip(items, refs)):
+        if kind == "f32":
+            assert_f32_output(it["y"].cpu().numpy(), ref, "%s problem %d" % (what, i))
+        else:
+            assert_bf16_output(bf16_host(it["y"]), ref, "%s problem %d" % (what, i))
+
+
+@pytest.mark.parametrize("layer", [0, 17])
+def test_batch_config2_layer(layer):
+    """A decode layer's seven projections (independent inputs) as one batch."""
+    items, refs = [], []
+    for p in WL.PROJECTIONS:
+        c = WL.config2_projection(layer, p.name)
+        P_d, beta, P_o, beta_o = both_pack(WL.master_weights(p.N, p.K, WL.master_seed(layer, p.name)))
+        refs.append(("bf16", O.f32_to_bf16(O.forward(c["x"], P_o, beta_o, gain=c["gain"],
+                                                     eps=WL.RMS_EPS, norm=True)["y"])))
+        items.append(dict(x=bf16_dev(c["x"]), gain=bf16_dev(c["gain"]), P=P_d, beta=beta,
+                          y=torch.empty((1, p.N), dtype=torch.bfloat16, device="cuda")))
+    B.bitlinear_forward_batch(B.make_batch(items), 1, WL.RMS_EPS)
+    _check_batch(items, refs, "config 2 layer %d batch" % layer)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5])
+def test_batch_mixed_problems(M):
+    specs = [(256, 128, True, torch.bfloat16, False), (2560, 640, False, torch.float32, False),
+             (6912, 2560, True, torch.bfloat16, True), (16, 4, False, torch.bfloat16, False),
+             (4096 + 16, 12, True, torch.float32, False)]
+    items, refs = _batch_case(specs, M, seed=5000 + M)
+    B.bitlinear_forward_batch(B.make_batch(items), M, WL.RMS_EPS)
+    _check_batch(items, refs, "mixed batch M=%d" % M)
+
+
+def test_batch_many_problems():
+    specs = [(16 * (1 + i % 7), 4 * (1 + i % 5), i % 2 == 0, torch.bfloat16, i % 3 == 0)
+             for i in range(40)]
+    items, refs = _batch_case(specs, 2, seed=7000)
+    B.bitlinear_forward_batch(B.make_batch(items), 2, WL.RMS_EPS)
+    _check_batch(items, refs, "40-problem batch")
+
+
+def test_quantized_batch_shared_input_qkv_and_gate_up():
+    """q|k|v share one quantised input, gate|up another: one launch each."""
+    for M in (1, 3, 6):
+        x = WL.activations(M, 2560, seed=8000 + M, outlier_frac=0.001)
+        g = WL.gain(2560, seed=8100)
+        q, s, rs = B.bitlinear_act_quant(bf16_dev(x), bf16_dev(g), WL.RMS_EPS)
+        for names in (("q", "k", "v"), ("gate", "up")):
+            items, refs = [], []
+            for name in names:
+                p = WL.PROJECTIONS[WL.PROJ_INDEX[name]]
+                P_d, beta, P_o, beta_o = both_pack(WL.master_weights(p.N, p.K,
+                                                                     WL.master_seed(3, name)))
+                refs.append(O.f32_to_bf16(O.forward(x, P_o, beta_o, gain=g, eps=WL.RMS_EPS,
+                                                    norm=True)["y"]))
+                items.append(dict(q=q, s_x=s, rowsum=rs, P=P_d, beta=beta,
+                                  y=torch.empty((M, p.N), dtype=torch.bfloat16, device="cuda")))
+            B.bitlinear_forward_quantized_batch(B.make_quantized_batch(items), M)
+            for it, ref, name in zip(items, refs, names):
+                assert_bf16_output(bf16_host(it["y"]), ref, "shared-input %s M=%d" % (name, M))
+
+
+def test_batch_of_many_tiny_problems_and_one_large():
+    """100 one-row problems land in the first CTA's byte range (more problems
+    than a CTA stages), next to a large one: both code paths in one launch."""
+    specs = [(16, 4, i % 2 == 0, torch.bfloat16, False) for i in range(100)]
+    specs.append((2560, 2560, True, torch.float32, False))
+    items, refs = _batch_case(specs, 1, seed=9000)
+    B.bitlinear_forward_batch(B.make_batch(items), 1, WL.RMS_EPS)
+    _check_batch(items, refs, "100 tiny + 1 large")
