@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the M=4096 prefill measurement reported beside the headline")
     return ap.parse_args()
 
 
@@ -259,6 +261,71 @@ class DecodeWorkload:
         return g
 
 
+class PrefillWorkload:
+    """Config-4 prefill: M=4096 tokens through gate, up, down, q, o (RMSNorm,
+    bf16 out).  Times the tensor-core GEMM launch on already-quantised codes and
+    the whole forward (quantise + GEMM)."""
+
+    def __init__(self, M=4096):
+        import ternary_weight_bitlinear_b200 as B
+        from ternary_weight_bitlinear_b200 import workloads as WL
+        self.B, self.WL, self.M = B, WL, M
+        self.items = []
+        for name in WL.CONFIG4_PROJECTIONS:
+            p = WL.PROJECTIONS[WL.PROJ_INDEX[name]]
+            W = torch.from_numpy(WL.master_weights(p.N, p.K, WL.master_seed(0, name))).cuda()
+            P, beta = B.bitlinear_pack(W)
+            del W
+            c = WL.config4_projection(name, M)
+            x = torch.from_numpy(c["x"].view(np.int16)).view(torch.bfloat16).cuda()
+            g = torch.from_numpy(c["gain"].view(np.int16)).view(torch.bfloat16).cuda()
+            q, sx, rs = B.bitlinear_act_quant(x, g, WL.RMS_EPS)
+            y = torch.empty((M, p.N), dtype=torch.bfloat16, device="cuda")
+            ws = torch.empty(B.bitlinear_forward_workspace_size(M, p.K, p.N), dtype=torch.uint8,
+                             device="cuda")
+            self.items.append(dict(name=name, K=p.K, N=p.N, P=P, beta=float(beta.item()), x=x,
+                                   g=g, q=q, sx=sx, rs=rs, y=y, ws=ws))
+
+    def gemm(self, it):
+        self.B.bitlinear_forward_quantized(it["q"], it["sx"], it["rs"], it["P"], it["beta"],
+                                           out=it["y"])
+
+    def forward(self, it):
+        self.B.bitlinear_forward(it["x"], it["P"], it["beta"], gain=it["g"], eps=self.WL.RMS_EPS,
+                                 out=it["y"], workspace=it["ws"])
+
+    def measure(self, reps, warmup, world):
+        peak, src = measured_int8_peak()
+        out = {"workload": "prefill M=4096: gate/up 2560->6912, down 6912->2560, q/o "
+                           "2560->2560; RMSNorm, bf16 out",
+               "int8_peak_tops": peak, "peak_source": src, "projections": {}}
+        tot_ops = tot_gemm_ms = tot_fwd_ms = 0.0
+        for it in self.items:
+            ops = 2.0 * self.M * it["N"] * it["K"]
+            ms_g = timed(lambda: self.gemm(it), reps, warmup, world) / reps
+            ms_f = timed(lambda: self.forward(it), reps, warmup, world) / reps
+            out["projections"][it["name"]] = {
+                "gemm_ms": ms_g, "gemm_tops": ops / ms_g / 1e9, "forward_ms": ms_f,
+                "frac_of_int8_peak": ops / ms_g / 1e9 / peak}
+            tot_ops += ops
+            tot_gemm_ms += ms_g
+            tot_fwd_ms += ms_f
+        out["gemm_tops"] = tot_ops / tot_gemm_ms / 1e9
+        out["frac_of_int8_peak"] = out["gemm_tops"] / peak
+        out["tokens_per_s"] = self.M / (tot_fwd_ms / 1000.0)  # one pass over the 5 projections
+        return out
+
+
+def measured_int8_peak():
+    """Dense int8 tensor peak: the measured bf16 GEMM burst x the nominal 2x ratio."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return 2.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 burst x 2 (nominal int8:bf16)"
+    except Exception:
+        return 2.0 * 1590.0, "fallback bf16 1.59 PF x 2"
+
+
 def timed(fn, steps, warmup, world):
     for _ in range(warmup):
         fn()
@@ -451,6 +518,11 @@ def main():
     ms_e2e = max_over_ranks(timed(e2e_step, args.steps, args.warmup, world), world)
     e2e_value = world * wl.M * args.steps / (ms_e2e / 1000.0)
 
+    prefill = None
+    if not args.no_prefill:
+        pw = PrefillWorkload()
+        prefill = pw.measure(max(3, min(args.steps, 20)), max(args.warmup, 2), world)
+
     status = wl.B.bitlinear_device_status()
     if status != 0:
         raise RuntimeError("device status %d after the timed region" % status)
@@ -474,6 +546,7 @@ def main():
                              "launch_us": gemv_launch_ms * 1000.0,
                              "bytes_per_launch": bytes_per_launch},
                 "variants": variants,
+                "prefill": prefill,
                 "e2e": {"value": e2e_value, "unit": "tokens/s",
                         "h2d_bytes_per_step": wl.h2d_bytes, "d2h_bytes_per_step": wl.d2h_bytes},
                 "gpu_launches": wl.launches["token_batch"] * args.steps,

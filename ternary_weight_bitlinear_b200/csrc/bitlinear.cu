@@ -14,6 +14,7 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "gemm_tc.cuh"
 #include "glue.cuh"
 #include "pack.cuh"
 #include "quant.cuh"
@@ -240,30 +241,101 @@ bl_status run_decode(const DecodeJob* jobs, int count, int mt, int dev, const De
     return launch_decode_cap<BL_MAX_BATCH>(jobs, count, mt, dev, info, stream);
 }
 
-// Matmul + epilogue on pre-quantised activations, any M: token groups of up
-// to four rows through the decode kernel.
+// ---- tensor-core GEMM (M > 4) ------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// 2-D uint8 tensor [outer, inner] (row stride = inner bytes), tiles of
+// box_outer x box_inner; elements outside the tensor read as zero.
+bool make_map_u8(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer,
+                 uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) {
+        snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled is unavailable");
+        return false;
+    }
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return false;
+    }
+    return true;
+}
+
+bl_status run_gemm(const int8_t* q, const float* s_x, const int32_t* rowsum, const uint8_t* P,
+                   float beta, int64_t M, int64_t K, int64_t N, void* y, int epi,
+                   const uint16_t* residual, int dev, const DeviceInfo& info,
+                   cudaStream_t stream) {
+    CUtensorMap map_q, map_p;
+    if (!make_map_u8(&map_q, q, (uint64_t)K, (uint64_t)M, kTcBK, kTcBM,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_u8(&map_p, P, (uint64_t)K, (uint64_t)(N / 4), kTcBK, kTcPackRows,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+        return BL_ERR_CUDA;
+    TcArgs a = {};
+    a.P = P;
+    a.s_x = s_x;
+    a.rowsum = rowsum;
+    a.y = y;
+    a.residual = residual;
+    a.beta = beta;
+    a.epi = epi;
+    a.M = (int)M;
+    a.K = (int)K;
+    a.R = (int)(N / 4);
+    a.N = N;
+    a.tiles_n = (int)((N / 4 + kTcPackRows - 1) / kTcPackRows);
+    a.tiles_m = (int)((M + kTcBM - 1) / kTcBM);
+    // 16-byte output accesses need every run of 32 outputs to start 16-byte aligned
+    const int64_t out_bytes = epi == kEpiBF16 ? 2 : 4;
+    a.vec_ok = ((N / 4) * out_bytes % 16 == 0) && (N * out_bytes % 16 == 0) &&
+               (reinterpret_cast<uintptr_t>(y) % 16 == 0) &&
+               (!residual || reinterpret_cast<uintptr_t>(residual) % 16 == 0);
+    if (prepare_kernel(reinterpret_cast<const void*>(gemm_tc_kernel), dev, info, kTcThreads,
+                       kTcSmemBytes) < 0)
+        return BL_ERR_CUDA;
+    const int64_t tiles = (int64_t)a.tiles_n * a.tiles_m;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(tiles, info.sms));
+    return launch(gemm_tc_kernel, dim3((unsigned)grid), dim3(kTcThreads), (size_t)kTcSmemBytes,
+                  stream, map_q, map_p, a);
+}
+
+// Matmul + epilogue on pre-quantised activations, any M: the decode kernel
+// for up to four tokens, the tensor-core GEMM beyond.
 bl_status run_quantized(const int8_t* q, const float* s_x, const int32_t* rowsum, const uint8_t* P,
                         float beta, int64_t M, int64_t K, int64_t N, void* y, int epi,
                         const uint16_t* residual, int dev, const DeviceInfo& info,
                         cudaStream_t stream) {
-    const size_t ysz = epi == kEpiBF16 ? 2 : 4;
-    for (int64_t m0 = 0; m0 < M; m0 += kDecMaxTokens) {
-        const int mt = (int)std::min<int64_t>(kDecMaxTokens, M - m0);
-        DecodeJob j;
-        j.q = q + m0 * K;
-        j.s_x = s_x ? s_x + m0 : nullptr;
-        j.rowsum = rowsum + m0;
-        j.P = P;
-        j.y = static_cast<char*>(y) + (size_t)(m0 * N) * ysz;
-        j.residual = residual ? residual + m0 * N : nullptr;
-        j.K = K;
-        j.N = N;
-        j.beta = beta;
-        j.epi = epi;
-        bl_status st = run_decode(&j, 1, mt, dev, info, stream);
-        if (st != BL_OK) return st;
-    }
-    return BL_OK;
+    if (M > kDecMaxTokens)
+        return run_gemm(q, s_x, rowsum, P, beta, M, K, N, y, epi, residual, dev, info, stream);
+    DecodeJob j = {q, s_x, rowsum, P, y, residual, K, N, beta, epi};
+    return run_decode(&j, 1, (int)M, dev, info, stream);
 }
 
 int epi_of(bl_out_dtype d) {

@@ -1,0 +1,395 @@
+// gemm_tc.cuh -- BitLinear matmul on the 5th-generation tensor cores (tcgen05),
+// for token counts beyond the decode kernel (prefill, batched decode).
+//
+// acc[m,n] = sum_k q[m,k] t[n,k] ("Transformers 实战 BitNet 1.58 位量化"
+// walkthrough, "推理侧 BitLinear": unpack_weights + F.linear) as a dense int8
+// contraction: D[m, n] = sum_k q[m,k] * code[n,k] with code = t + 1 in {0,1,2},
+// then acc = D - rowsum_q[m] (exact), rescaled like the decode kernel.
+//
+// Tile: 128 tokens x 256 output rows (= 64 packed rows x 4 bit pairs), K in
+// stages of 128 bytes.  Persistent CTAs, one per SM, walk the tiles
+// round-robin.  Warp roles:
+//   warp 0      TMA producer: per stage, the 128x128-byte int8 activation tile
+//               (A operand, 128-byte swizzle, rows past M zero-filled) and the
+//               64x128-byte packed weight tile; no multicast.
+//   warps 1-4   expansion: 2-bit codes -> int8 codes written straight into the
+//               128-byte-swizzled K-major B operand (256 rows) in shared memory.
+//   warp 5      one thread issues tcgen05.mma.cta_group::1.kind::i8
+//               (M=128, N=256, K=32) into a TMEM accumulator (2 buffers).
+//   warps 6-9   epilogue: each thread owns one token (a TMEM lane of its
+//               warp's quadrant) and 256 output rows: tcgen05.ld, minus the
+//               token's row sum, rescale, 16-byte stores of contiguous outputs.
+// Loads run up to kTcStages stages ahead; expanded operands are double-buffered.
+// Every mbarrier wait is bounded (records BL_ERR_TIMEOUT and unwinds).
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "decode.cuh"
+
+namespace bl {
+
+constexpr int kTcBM = 128;        // tokens per tile (MMA M)
+constexpr int kTcBN = 256;        // output rows per tile (MMA N)
+constexpr int kTcBK = 128;        // K bytes per stage (one 128-byte swizzle atom)
+constexpr int kTcPackRows = 64;   // packed rows per tile (x 4 bit pairs = kTcBN)
+constexpr int kTcStages = 5;      // load stages (A + packed weights)
+constexpr int kTcExp = 2;         // expanded-B buffers
+constexpr int kTcThreads = 320;
+constexpr int kTcEpiWarp0 = 6;
+constexpr int kTcABytes = kTcBM * kTcBK;          // 16 KB activations
+constexpr int kTcBBytes = kTcBN * kTcBK;          // 32 KB expanded codes
+constexpr int kTcPBytes = kTcPackRows * kTcBK;    // 8 KB packed codes
+constexpr int kTcStageTx = kTcABytes + kTcPBytes;
+// layout from a 1024-aligned base: A[5] | B[2] | P[5] | barriers | tmem addr
+constexpr int kTcOffB = kTcStages * kTcABytes;
+constexpr int kTcOffP = kTcOffB + kTcExp * kTcBBytes;
+constexpr int kTcOffBar = kTcOffP + kTcStages * kTcPBytes;
+constexpr int kTcNumBars = 2 * kTcStages + 2 * kTcExp + 5;
+constexpr int kTcOffTmem = kTcOffBar + 8 * kTcNumBars;
+constexpr int kTcSmemBytes = kTcOffTmem + 16 + 1024;   // + alignment slack
+constexpr uint32_t kTcTmemCols = 2 * kTcBN;           // two accumulators
+static_assert(kTcSmemBytes <= 227 * 1024, "shared memory budget");
+
+struct TcArgs {
+    const uint8_t* P;          // [R,K] (through tmap_p)
+    const float* s_x;          // [M]
+    const int32_t* rowsum;     // [M]
+    void* y;                   // [M,N]
+    const uint16_t* residual;  // bf16 [M,N] or nullptr
+    float beta;
+    int epi;
+    int M;
+    int K;
+    int R;
+    int64_t N;
+    int tiles_n;               // ceil(R / 64)
+    int tiles_m;               // ceil(M / 128)
+    int vec_ok;                // outputs of 32 consecutive rows can use 16-byte accesses
+};
+
+// ---- tcgen05 / TMA wrappers ------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(dst_smem), "r"(cols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, int8 x int8 -> int32.
+__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on `bar` once every tcgen05 op this thread issued so far completes.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(bar) : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+        " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31},"
+        " [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (stride byte offset), descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor: int32 accumulate, signed 8-bit A and B, both
+// K-major, M = kTcBM, N = kTcBN.
+constexpr uint32_t kTcIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTcBN >> 3) << 17) |
+                              ((uint32_t)(kTcBM >> 4) << 24);
+
+// Byte offset of the 16-byte chunk `chunk16` of `row` in a 128-byte-wide,
+// 128-byte-swizzled K-major tile (8-row groups of 1024 bytes).
+__device__ __forceinline__ uint32_t sw128_offset(int row, int chunk16) {
+    return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((chunk16 ^ (row & 7)) << 4));
+}
+
+// Store 32 consecutive outputs y[m, n0 .. n0+31] of one token (scalar path:
+// only rows < R, i.e. n0 + j with j < valid).
+__device__ __forceinline__ float tc_scale(int acc, float beta, float s_x) {
+    return __fdiv_rn(__fmul_rn(__int2float_rn(acc), beta), s_x);
+}
+
+__device__ __forceinline__ void tc_store_row32(const TcArgs& a, int64_t base, const uint32_t (&v)[32], int rsum,
+                               float s_x, int valid) {
+    if (a.vec_ok && valid == 32) {
+        if (a.epi == kEpiBF16) {
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                uint32_t lo = float_to_bf16_bits(tc_scale((int)v[2 * j] - rsum, a.beta, s_x));
+                uint32_t hi = float_to_bf16_bits(tc_scale((int)v[2 * j + 1] - rsum, a.beta, s_x));
+                w[j] = lo | (hi << 16);
+            }
+            if (a.residual) {
+                const uint4* rp = reinterpret_cast<const uint4*>(a.residual + base);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 r = __ldcg(rp + c);
+                    const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const uint32_t x = w[4 * c + h];
+                        const uint32_t lo = float_to_bf16_bits(__fadd_rn(
+                            bf16_bits_to_float(rr[h] & 0xFFFFu), bf16_bits_to_float(x & 0xFFFFu)));
+                        const uint32_t hi = float_to_bf16_bits(__fadd_rn(
+                            bf16_bits_to_float(rr[h] >> 16), bf16_bits_to_float(x >> 16)));
+                        w[4 * c + h] = lo | (hi << 16);
+                    }
+                }
+            }
+            uint4* yp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.y) + base);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) yp[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        } else {
+            uint4* yp = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.y) + base);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t w[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int acc = (int)v[4 * c + h] - rsum;
+                    w[h] = a.epi == kEpiI32 ? (uint32_t)acc : __float_as_uint(tc_scale(acc, a.beta, s_x));
+                }
+                yp[c] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        return;
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        if (j >= valid) break;
+        const int acc = (int)v[j] - rsum;
+        const int64_t idx = base + j;
+        if (a.epi == kEpiI32) {
+            static_cast<int32_t*>(a.y)[idx] = acc;
+        } else if (a.epi == kEpiF32) {
+            static_cast<float*>(a.y)[idx] = tc_scale(acc, a.beta, s_x);
+        } else {
+            uint16_t b = float_to_bf16_bits(tc_scale(acc, a.beta, s_x));
+            if (a.residual)
+                b = float_to_bf16_bits(
+                    __fadd_rn(bf16_bits_to_float(__ldcg(a.residual + idx)), bf16_bits_to_float(b)));
+            static_cast<uint16_t*>(a.y)[idx] = b;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
+    const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_p,
+    const TcArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;  // 1024-aligned for the 128-byte swizzle
+    uint8_t* sm = smem_raw + (base - raw);
+    const uint32_t sA = base, sB = base + kTcOffB, sP = base + kTcOffP;
+    const uint32_t bars = base + kTcOffBar;
+    auto full_bar = [&](int s) { return bars + 8u * s; };
+    auto empty_bar = [&](int s) { return bars + 8u * (kTcStages + s); };
+    auto bready_bar = [&](int e) { return bars + 8u * (2 * kTcStages + e); };
+    auto bfree_bar = [&](int e) { return bars + 8u * (2 * kTcStages + kTcExp + e); };
+    auto accfull_bar = [&](int b) { return bars + 8u * (2 * kTcStages + 2 * kTcExp + b); };
+    auto accempty_bar = [&](int b) { return bars + 8u * (2 * kTcStages + 2 * kTcExp + 2 + b); };
+    const uint32_t mma_done_bar = bars + 8u * (2 * kTcStages + 2 * kTcExp + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kTcOffTmem);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int e = 0; e < kTcExp; ++e) {
+            mbar_init(bready_bar(e), 4);
+            mbar_init(bfree_bar(e), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(accfull_bar(b), 1);
+            mbar_init(accempty_bar(b), 4);
+        }
+        mbar_init(mma_done_bar, 1);
+        mbar_init_fence();
+    }
+    if (warp == 5) tmem_alloc(smem_addr(tmem_slot), kTcTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    pdl_wait();
+    pdl_launch_dependents();
+
+    const int64_t tiles = (int64_t)a.tiles_n * a.tiles_m;
+    const int kstages = (a.K + kTcBK - 1) / kTcBK;
+    bool ok = true;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            uint32_t g = 0;
+            uint32_t inflight_from = 0;  // stages [inflight_from, g) may still be landing
+            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int tn = (int)(t / a.tiles_m), tm = (int)(t % a.tiles_m);
+                for (int ks = 0; ks < kstages; ++ks, ++g) {
+                    const int s = (int)(g % kTcStages);
+                    if (!mbar_wait(empty_bar(s), ((g / kTcStages) & 1u) ^ 1u)) { ok = false; break; }
+                    inflight_from = g >= kTcStages ? g - kTcStages + 1 : 0;
+                    mbar_arrive_expect_tx(full_bar(s), kTcStageTx);
+                    tma_load_2d(sA + s * kTcABytes, &tmap_q, ks * kTcBK, tm * kTcBM, full_bar(s));
+                    tma_load_2d(sP + s * kTcPBytes, &tmap_p, ks * kTcBK, tn * kTcPackRows, full_bar(s));
+                }
+            }
+            // after a failed wait, let the copies still in flight land first
+            if (!ok)
+                for (uint32_t j = inflight_from; j < g; ++j)
+                    mbar_wait(full_bar((int)(j % kTcStages)), (j / kTcStages) & 1u);
+        }
+    } else if (warp >= 1 && warp <= 4) {
+        // ---------------- expansion: 2-bit codes -> int8 B tile ----------------
+        const int e0 = threadIdx.x - 32;  // 0..127
+        uint32_t g = 0;
+        for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            for (int ks = 0; ks < kstages; ++ks, ++g) {
+                const int s = (int)(g % kTcStages), e = (int)(g % kTcExp);
+                const bool got = mbar_wait(full_bar(s), (g / kTcStages) & 1u) &&
+                                 mbar_wait(bfree_bar(e), ((g / kTcExp) & 1u) ^ 1u);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                const uint8_t* pk = sm + kTcOffP + s * kTcPBytes;
+                uint8_t* bt = sm + kTcOffB + e * kTcBBytes;
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int item = e0 + it * 128;  // (packed row, 16-byte chunk)
+                    const int rr = item >> 3, ch = item & 7;
+                    const uint4 w = *reinterpret_cast<const uint4*>(pk + rr * kTcBK + ch * 16);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = i * kTcPackRows + rr;
+                        const uint4 c = make_uint4((w.x >> (2 * i)) & 0x03030303u,
+                                                   (w.y >> (2 * i)) & 0x03030303u,
+                                                   (w.z >> (2 * i)) & 0x03030303u,
+                                                   (w.w >> (2 * i)) & 0x03030303u);
+                        *reinterpret_cast<uint4*>(bt + sw128_offset(row, ch)) = c;
+                    }
+                }
+                fence_proxy_async_smem();  // generic writes -> visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bready_bar(e));
+            }
+        }
+    } else if (warp == 5) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            uint32_t g = 0, tl = 0;
+            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tl) {
+                const int buf = (int)(tl & 1);
+                if (!mbar_wait(accempty_bar(buf), ((tl >> 1) & 1u) ^ 1u)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(buf * kTcBN);
+                for (int ks = 0; ks < kstages; ++ks, ++g) {
+                    const int s = (int)(g % kTcStages), e = (int)(g % kTcExp);
+                    if (!mbar_wait(full_bar(s), (g / kTcStages) & 1u) ||
+                        !mbar_wait(bready_bar(e), (g / kTcExp) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc_sw128(sA + s * kTcABytes);
+                    const uint64_t bd = smem_desc_sw128(sB + e * kTcBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kTcBK / 32; ++kk)  // +32 bytes = +2 in the address field
+                        tc_mma_i8(d, ad + 2u * kk, bd + 2u * kk, kTcIdesc, (ks | kk) != 0);
+                    tc_commit(empty_bar(s));  // activation + packed stage reusable
+                    tc_commit(bfree_bar(e));  // expanded operand reusable
+                }
+                if (!ok) break;
+                tc_commit(accfull_bar(buf));  // accumulator ready for the epilogue
+            }
+            // every MMA this thread issued has finished before TMEM is freed
+            tc_commit(mma_done_bar);
+            mbar_wait(mma_done_bar, 0);
+        }
+    } else {
+        // ---------------- epilogue: one token per thread ----------------
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        uint32_t tl = 0;
+        for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tl) {
+            const int tn = (int)(t / a.tiles_m), tm = (int)(t % a.tiles_m);
+            const int buf = (int)(tl & 1);
+            const int m = tm * kTcBM + q * 32 + lane;  // this thread's token
+            const bool live = m < a.M;
+            const float sx = (live && a.epi != kEpiI32) ? __ldcg(a.s_x + m) : 1.0f;
+            const int rsum = live ? __ldcg(a.rowsum + m) : 0;
+            const bool got = mbar_wait(accfull_bar(buf), (tl >> 1) & 1u);
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kTcBN);
+#pragma unroll 1
+            for (int c0 = 0; c0 < kTcBN; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(taddr + (uint32_t)c0, v);
+                const int i = c0 / kTcPackRows;                       // bit pair
+                const int r = tn * kTcPackRows + (c0 % kTcPackRows);  // first packed row
+                const int valid = min(32, a.R - r);
+                if (live && valid > 0)
+                    tc_store_row32(a, (int64_t)m * a.N + (int64_t)i * a.R + r, v, rsum, sx, valid);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(accempty_bar(buf));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTcTmemCols);
+    }
+}
+
+}  // namespace bl

@@ -345,3 +345,37 @@ def test_batch_of_many_tiny_problems_and_one_large():
     items, refs = _batch_case(specs, 1, seed=9000)
     B.bitlinear_forward_batch(B.make_batch(items), 1, WL.RMS_EPS)
     _check_batch(items, refs, "100 tiny + 1 large")
+
+
+# ---------------------------------------------------------------------------
+# tensor-core GEMM path (M > 4): ragged tiles, store paths, persistent loop
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("M,K,N,out,residual", [
+    (5, 16, 4, "f32", False),          # everything smaller than one tile
+    (129, 272, 36, "f32", False),      # token tile + 1, K not a multiple of 128, R=9
+    (300, 4112, 12, "bf16", True),     # R=3: scalar store path with residual
+    (257, 128, 256, "bf16", False),    # exactly one K stage, one weight tile
+    (1000, 2560, 6912, "bf16", True),  # 216 tiles > 148 CTAs: both accumulators reused
+    (130, 6912, 2560, "i32", False),   # exact int32 accumulators, 54 K stages
+])
+def test_gemm_path_shapes(M, K, N, out, residual):
+    x = special_rows(WL.activations(M, K, seed=M * 7 + K, row_std=(0.1, 10.0)))
+    W = WL.master_weights(N, K, seed=N * 3 + K)
+    P_d, beta, P_o, beta_o = both_pack(W)
+    q, s, rs = B.bitlinear_act_quant(bf16_dev(x))
+    q_o, s_o, rs_o = O.quantize_input(x)
+    assert_exact(q.cpu().numpy(), q_o, "codes")
+    if out == "i32":
+        acc = B.bitlinear_accumulate(q, rs, P_d)
+        assert_exact(acc.cpu().numpy(), O.ternary_matmul(q_o, O.unpack(P_o)), "int32 accumulators")
+        return
+    y_o = O.forward(x, P_o, beta_o)["y"]
+    if out == "f32":
+        y = B.bitlinear_forward_quantized(q, s, rs, P_d, beta, out_dtype=torch.float32)
+        assert_f32_output(y.cpu().numpy(), y_o, "gemm f32")
+    else:
+        r = WL.activations(M, N, seed=M + N) if residual else None
+        y = bf16_dev(r) if residual else torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        B.bitlinear_forward_quantized(q, s, rs, P_d, beta, residual=y if residual else None, out=y)
+        ref = O.residual_add(r, O.f32_to_bf16(y_o)) if residual else O.f32_to_bf16(y_o)
+        assert_bf16_output(bf16_host(y), ref, "gemm bf16")
