@@ -25,6 +25,7 @@ using namespace bl;
 
 constexpr int kQuantThreads = 256;
 constexpr int kSmallBatch = 8;  // parameter-table size of small batches
+constexpr int64_t kQuantWarpMinRows = 1024;  // rows from which a warp per row pays off
 
 // ---- device properties and per-kernel launch settings ---------------------
 struct DeviceInfo {
@@ -160,6 +161,18 @@ bl_status launch_quant_cap(const QuantProblem* probs, int count, int64_t M, floa
     for (int i = 0; i < count; ++i) {
         b.p[i] = probs[i];
         kmax = std::max(kmax, probs[i].K);
+    }
+    if (kmax <= kQuantWarpMaxK && (int64_t)count * M >= kQuantWarpMinRows) {
+        // many rows (prefill): one warp per row, up to 8 rows per CTA; few rows
+        // (decode) go to one CTA per row below, which has the lower latency
+        const int wpb = (int)std::max<int64_t>(1, std::min<int64_t>(8, 65536 / (4 * (int64_t)kmax)));
+        auto fn = quant_warp_kernel<CAP>;
+        const int64_t smem = (int64_t)wpb * 4 * kmax;
+        if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, 32 * wpb, smem) < 0)
+            return BL_ERR_CUDA;
+        const int64_t rows = (int64_t)count * M;
+        return launch(fn, dim3((unsigned)((rows + wpb - 1) / wpb)), dim3(32 * wpb), (size_t)smem,
+                      stream, b, kmax);
     }
     auto fn = quant_batch_kernel<kQuantThreads, CAP>;
     const int64_t smem = 2 * (int64_t)kmax;  // the staged bf16 row

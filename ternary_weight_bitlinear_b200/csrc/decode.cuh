@@ -39,7 +39,8 @@ namespace bl {
 constexpr int kDecThreads = 512;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kDecSlots = 8;          // copies in flight per warp (one mbarrier each)
-constexpr int kDecChunk = 4096;       // largest single copy: a row, or a piece of a long row
+constexpr int kDecChunk = 5120;       // largest single copy: 1-2 rows, or a piece of a long row
+constexpr int kDecMaxRows = 2;        // rows per copy (one per half-warp)
 constexpr int kDecRing = 10240;       // bytes of each warp's ring of copies
 constexpr int kDecMaxTokens = 4;
 constexpr int kDecQBudget = 48 * 1024;  // shared-memory bytes for staged codes
@@ -53,11 +54,13 @@ constexpr int kDecMetaBytes = kDecMaxStaged * kDecMaxTokens * 8 + kDecMaxStaged 
 // Per-warp queue of the descriptors of copies in flight (issued, not consumed).
 struct ItemDesc {
     int p;          // problem
-    int r;          // row
-    int c;          // chunk of the row
+    int r;          // first row
+    int c;          // chunk of the row (rows longer than kDecChunk)
     int bytes;
     uint32_t at;    // ring offset
     uint32_t used;  // ring bytes it holds (skipped tail + bytes)
+    int rows;       // whole rows in the copy (1 or 2; 1 for a chunk)
+    int pad;
 };
 constexpr int kDecDescBytes = kDecWarps * kDecSlots * (int)sizeof(ItemDesc);
 constexpr int kDecSmemBytes =
@@ -138,15 +141,23 @@ struct Walker {
         settle(b, hi);
     }
     __device__ __forceinline__ bool valid(const DecBatch<CAP>& b) const { return p < b.count; }
-    __device__ __forceinline__ int bytes() const { return min(kDecChunk, K - c * kDecChunk); }
-    __device__ __forceinline__ bool last_chunk() const { return (c + 1) * kDecChunk >= K; }
+    // whole rows in the next copy (short rows are copied two at a time)
+    __device__ __forceinline__ int rows() const {
+        return K <= kDecChunk ? min(min(kDecMaxRows, kDecChunk / K), r_end - r) : 1;
+    }
+    __device__ __forceinline__ int bytes() const {
+        return K <= kDecChunk ? rows() * K : min(kDecChunk, K - c * kDecChunk);
+    }
+    __device__ __forceinline__ bool last_chunk() const {
+        return K <= kDecChunk || (c + 1) * kDecChunk >= K;
+    }
     __device__ __forceinline__ const uint8_t* src() const {
         return P + (int64_t)r * K + c * kDecChunk;
     }
     __device__ __forceinline__ void advance(const DecBatch<CAP>& b, int64_t hi) {
         if (!last_chunk()) { ++c; return; }
+        r += rows();
         c = 0;
-        ++r;
         settle(b, hi);
     }
 };
@@ -209,6 +220,21 @@ __device__ __forceinline__ int warp_reduce4(const int (&a)[4], int lane) {
     return k;
 }
 
+// The same within each half-warp: on return lane 16h + 4i holds the total of
+// a[i] over lanes 16h .. 16h+15 (5 shuffles for both halves at once).
+__device__ __forceinline__ int half_reduce4(const int (&a)[4], int lane) {
+    const bool hi8 = lane & 8, hi4 = lane & 4;
+    int k0 = hi8 ? a[2] : a[0], k1 = hi8 ? a[3] : a[1];
+    const int s0 = hi8 ? a[0] : a[2], s1 = hi8 ? a[1] : a[3];
+    k0 += __shfl_xor_sync(0xffffffffu, s0, 8);
+    k1 += __shfl_xor_sync(0xffffffffu, s1, 8);
+    int k = hi4 ? k1 : k0;
+    k += __shfl_xor_sync(0xffffffffu, hi4 ? k0 : k1, 4);
+    k += __shfl_xor_sync(0xffffffffu, k, 2);
+    k += __shfl_xor_sync(0xffffffffu, k, 1);
+    return k;
+}
+
 template <int MT, int CAP>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
     const __grid_constant__ DecBatch<CAP> b) {
@@ -253,7 +279,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
             if (spot.used > ring_free) break;
             const uint32_t bar = bar0 + 8u * (issued % kDecSlots);
             if (lane == 0) {
-                my_descs[issued % kDecSlots] = ItemDesc{iw.p, iw.r, iw.c, bytes, spot.at, spot.used};
+                my_descs[issued % kDecSlots] =
+                    ItemDesc{iw.p, iw.r, iw.c, bytes, spot.at, spot.used, iw.rows(), 0};
                 fence_proxy_async_smem();  // this warp's earlier reads of the ring come first
                 mbar_arrive_expect_tx(bar, (uint32_t)bytes);
                 bulk_g2s_stream(smem_addr(ring + spot.at), iw.src(), (uint32_t)bytes, bar, policy);
@@ -337,39 +364,76 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
         }
         const bool got = mbar_wait(bar0 + 8u * (done % kDecSlots), (done / kDecSlots) & 1u);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        const uint4* wp = reinterpret_cast<const uint4*>(ring + d.at);
-        const int nvec = d.bytes >> 4;
+        const uint8_t* wbase = ring + d.at;
         const int8_t* qrow = qbase + d.c * kDecChunk;
-        if (staged) {
+        if (d.rows == 2) {
+            // two rows: half-warp h takes row d.r + h
+            const int h = lane >> 4, hl = lane & 15;
+            const uint4* wp = reinterpret_cast<const uint4*>(wbase + h * K);
+            const int nvec = K >> 4;
+            if (staged) {
 #pragma unroll 4
-            for (int v = lane; v < nvec; v += 32) {
-                const uint4 w4 = wp[v];
+                for (int v = hl; v < nvec; v += 16) {
+                    const uint4 w4 = wp[v];
 #pragma unroll
-                for (int m = 0; m < MT; ++m)
-                    dot16(w4, reinterpret_cast<const uint4*>(qrow + m * K)[v], acc[m]);
+                    for (int m = 0; m < MT; ++m)
+                        dot16(w4, reinterpret_cast<const uint4*>(qrow + m * K)[v], acc[m]);
+                }
+            } else {
+                for (int v = hl; v < nvec; v += 16) {
+                    const uint4 w4 = wp[v];
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+                        dot16(w4, __ldcg(reinterpret_cast<const uint4*>(qrow + (int64_t)m * K) + v),
+                              acc[m]);
+                }
             }
         } else {
-            for (int v = lane; v < nvec; v += 32) {
-                const uint4 w4 = wp[v];
+            const uint4* wp = reinterpret_cast<const uint4*>(wbase);
+            const int nvec = d.bytes >> 4;
+            if (staged) {
+#pragma unroll 4
+                for (int v = lane; v < nvec; v += 32) {
+                    const uint4 w4 = wp[v];
 #pragma unroll
-                for (int m = 0; m < MT; ++m)
-                    dot16(w4, __ldcg(reinterpret_cast<const uint4*>(qrow + (int64_t)m * K) + v),
-                          acc[m]);
+                    for (int m = 0; m < MT; ++m)
+                        dot16(w4, reinterpret_cast<const uint4*>(qrow + m * K)[v], acc[m]);
+                }
+            } else {
+                for (int v = lane; v < nvec; v += 32) {
+                    const uint4 w4 = wp[v];
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+                        dot16(w4, __ldcg(reinterpret_cast<const uint4*>(qrow + (int64_t)m * K) + v),
+                              acc[m]);
+                }
             }
         }
         __syncwarp();
         ring_free += d.used;
         ++done;
         refill();
-        if ((d.c + 1) * kDecChunk >= K) {  // last chunk of the row: reduce and store
+        if ((d.c + 1) * kDecChunk >= K || d.rows == 2) {  // the item ends its row(s)
             const DecProblem& pr = b.p[cur_p];
+            if (d.rows == 2) {
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                const int tot = warp_reduce4(acc[m], lane);
-                if ((lane & 7) == 0) {
-                    const int i = lane >> 3;
-                    store_output(pr, (int64_t)m * pr.N + (int64_t)i * pr.R + d.r,
-                                 (tot >> (2 * i)) - rsum[m], sx[m]);
+                for (int m = 0; m < MT; ++m) {
+                    const int tot = half_reduce4(acc[m], lane);
+                    if ((lane & 3) == 0) {
+                        const int i = (lane >> 2) & 3;
+                        store_output(pr, (int64_t)m * pr.N + (int64_t)i * pr.R + d.r + (lane >> 4),
+                                     (tot >> (2 * i)) - rsum[m], sx[m]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    const int tot = warp_reduce4(acc[m], lane);
+                    if ((lane & 7) == 0) {
+                        const int i = lane >> 3;
+                        store_output(pr, (int64_t)m * pr.N + (int64_t)i * pr.R + d.r,
+                                     (tot >> (2 * i)) - rsum[m], sx[m]);
+                    }
                 }
             }
         }

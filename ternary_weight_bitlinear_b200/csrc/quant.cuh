@@ -4,8 +4,11 @@
 // "BitLinear 的三步量化", step 3 (per-token absmax to [-128,127], scale
 // 127/max clamped at 1e-5) and the forward order of section "推理侧 BitLinear"
 // (RMSNorm first when present).  The norm formula is the standard RMSNorm with
-// the sum of squares taken exactly (binary64 with error-free TwoSum, fixed
-// reduction order), so r = RN32(1/sqrt(SS/K + eps)) is reproducible bit for bit.
+// the sum of squares rounded once from its exact value, so
+// r = RN32(1/sqrt(SS/K + eps)) is reproducible bit for bit: a one-FMA-per-element
+// binary64 sum with a rigorous error interval decides r whenever both ends of
+// the interval give the same binary32 value, else (rarely) the sum is redone
+// with error-free TwoSum accumulation.
 //
 // One CTA works on one token row; all loads are 16-byte vectors (8 bf16).  The
 // row is read from global memory once and staged in shared memory.
@@ -95,6 +98,31 @@ __device__ __forceinline__ float norm_elem(float x, float r, float g) {
     return __fmul_rn(__fmul_rn(x, r), g);
 }
 
+// r = RN32(1 / sqrt(RN64(SS/K) + eps)), each step a binary64 IEEE operation.
+// Non-increasing in ss.
+__device__ __forceinline__ float rms_factor(double ss, int K, float eps) {
+    const double ms = __ddiv_rn(ss, (double)K);
+    const double var = __dadd_rn(ms, (double)eps);
+    const double sd = __dsqrt_rn(var);
+    return __double2float_rn(__ddiv_rn(1.0, sd));
+}
+
+// Fast path for the factor: `approx` is a plain binary64 sum, in any order, of
+// the K exact squares (non-negative), so the exact sum lies within a relative
+// (K + 64) * 2^-52 of it (twice the textbook bound).  rms_factor is monotone,
+// so if both ends of that interval (computed with directed rounding) give the
+// same binary32 value, it is the value of the exactly rounded sum.  Returns
+// false when the ends differ and the exact sum is needed.
+__device__ __forceinline__ bool rms_factor_bounded(double approx, int K, float eps, float& r) {
+    const double delta = (double)(K + 64) * 0x1p-52;
+    const double lo = __dmul_rd(approx, __dsub_rd(1.0, delta));
+    const double hi = __dmul_ru(approx, __dadd_ru(1.0, delta));
+    const float r_small = rms_factor(hi, K, eps);
+    const float r_large = rms_factor(lo, K, eps);
+    r = r_small;
+    return r_small == r_large;
+}
+
 // Quantise one token row.  x: K bf16 (global, 16-byte aligned), read once
 // with ld.global.cg (it may have just been written by the previous kernel) and
 // staged in xs (shared, K/8 vectors); gain: K bf16 or nullptr (no norm); q: K
@@ -112,24 +140,31 @@ __device__ void quantize_row(const uint16_t* __restrict__ x, const uint16_t* __r
     float r = 1.0f;
     float mx = 0.0f;
     if (norm) {
-        double hi = 0.0, lo = 0.0;
+        double ss = 0.0;  // plain binary64 sum of the exact squares
         for (int v = threadIdx.x; v < nvec; v += NT) {
             const uint4 u = __ldcg(xv + v);
             xs[v] = u;
             float f[8];
             unpack8_bf16(u, f);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const double d = (double)f[j];
-                dd_add(hi, lo, __dmul_rn(d, d));  // exact square of a bf16 value
-            }
+            for (int j = 0; j < 8; ++j) ss = __fma_rn((double)f[j], (double)f[j], ss);
         }
-        const double ss = block_sum_dd<NT>(hi, lo, sc);
-        const double ms = __ddiv_rn(ss, (double)K);
-        const double var = __dadd_rn(ms, (double)eps);
-        const double sd = __dsqrt_rn(var);
-        const double rd = __ddiv_rn(1.0, sd);
-        r = __double2float_rn(rd);
+        const double approx = block_sum_dd<NT>(ss, 0.0, sc);
+        if (!rms_factor_bounded(approx, K, eps, r)) {
+            // rare: the interval straddles a rounding boundary; take the sum exactly
+            __syncthreads();
+            double hi = 0.0, lo = 0.0;
+            for (int v = threadIdx.x; v < nvec; v += NT) {
+                float f[8];
+                unpack8_bf16(xs[v], f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const double d = (double)f[j];
+                    dd_add(hi, lo, __dmul_rn(d, d));  // exact square of a bf16 value
+                }
+            }
+            r = rms_factor(block_sum_dd<NT>(hi, lo, sc), K, eps);
+        }
         for (int v = threadIdx.x; v < nvec; v += NT) {
             float f[8], g[8];
             unpack8_bf16(xs[v], f);
@@ -207,6 +242,140 @@ __global__ void __launch_bounds__(NT) quant_batch_kernel(const __grid_constant__
     quantize_row<NT>(pr.x + (int64_t)m * pr.K, pr.gain, b.eps, pr.K, pr.q + (int64_t)m * pr.K, xs,
                      sc, s, rs);
     if (threadIdx.x == 0) {
+        pr.s_x[m] = s;
+        if (pr.rowsum) pr.rowsum[m] = rs;
+    }
+}
+
+// ---- one warp per (problem, token row): no block-wide barriers ---------------
+constexpr int kQuantWarpMaxK = 16384;  // the row is staged in the warp's own shared memory
+
+// Deterministic warp sum of (hi, lo) pairs (fixed shuffle tree; every lane
+// ends with the same value: the partner order is the same on both sides).
+__device__ __forceinline__ double warp_sum_dd(double hi, double lo) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double ohi = __shfl_down_sync(0xffffffffu, hi, o);
+        const double olo = __shfl_down_sync(0xffffffffu, lo, o);
+        if (lane < o) dd_merge(hi, lo, ohi, olo);
+    }
+    hi = __shfl_sync(0xffffffffu, hi, 0);
+    lo = __shfl_sync(0xffffffffu, lo, 0);
+    return __dadd_rn(hi, lo);
+}
+
+// Quantise one token row with one warp (same arithmetic as quantize_row).  The
+// row and its gain are first copied into the warp's shared memory (xs, gs:
+// K/8 vectors each) with every 16-byte copy in flight at once.
+__device__ void quantize_row_warp(const uint16_t* __restrict__ x, const uint16_t* __restrict__ gain,
+                                  float eps, int K, int8_t* __restrict__ q, uint4* __restrict__ xs,
+                                  uint4* __restrict__ gs, float& s_out, int& rowsum_out) {
+    const int lane = threadIdx.x & 31;
+    const int nvec = K >> 3;
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    const uint4* gv = reinterpret_cast<const uint4*>(gain);
+    const bool norm = gain != nullptr;
+    for (int v = lane; v < nvec; v += 32) cp_async16(xs + v, xv + v);
+    if (norm)
+        for (int v = lane; v < nvec; v += 32) cp_async16(gs + v, gv + v);
+    cp_async_wait_all();
+    __syncwarp();
+
+    float r = 1.0f;
+    float mx = 0.0f;
+    if (norm) {
+        double ss0 = 0.0, ss1 = 0.0;  // plain binary64 sums of the exact squares
+        for (int v = lane; v < nvec; v += 32) {
+            float f[8];
+            unpack8_bf16(xs[v], f);
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                ss0 = __fma_rn((double)f[j], (double)f[j], ss0);
+                ss1 = __fma_rn((double)f[j + 1], (double)f[j + 1], ss1);
+            }
+        }
+        const double approx = warp_sum_dd(__dadd_rn(ss0, ss1), 0.0);
+        if (!rms_factor_bounded(approx, K, eps, r)) {
+            // rare: the interval straddles a rounding boundary; take the sum exactly
+            double hi[8], lo[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) hi[j] = lo[j] = 0.0;
+            for (int v = lane; v < nvec; v += 32) {
+                float f[8];
+                unpack8_bf16(xs[v], f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const double d = (double)f[j];
+                    dd_add(hi[j], lo[j], __dmul_rn(d, d));  // exact square of a bf16 value
+                }
+            }
+#pragma unroll
+            for (int j = 1; j < 8; ++j) dd_merge(hi[0], lo[0], hi[j], lo[j]);
+            r = rms_factor(warp_sum_dd(hi[0], lo[0]), K, eps);
+        }
+        for (int v = lane; v < nvec; v += 32) {
+            float f[8], g[8];
+            unpack8_bf16(xs[v], f);
+            unpack8_bf16(gs[v], g);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(norm_elem(f[j], r, g[j])));
+        }
+    } else {
+        for (int v = lane; v < nvec; v += 32) {
+            float f[8];
+            unpack8_bf16(xs[v], f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(f[j]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float s = __fdiv_rn(127.0f, fmaxf(mx, kScaleFloor));
+
+    int rs = 0;
+    for (int v = lane; v < nvec; v += 32) {
+        float f[8], g[8];
+        unpack8_bf16(xs[v], f);
+        if (norm) {
+            unpack8_bf16(gs[v], g);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] = norm_elem(f[j], r, g[j]);
+        }
+        uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            int c = __float2int_rn(__fmul_rn(f[j], s));  // round half to even
+            c = min(max(c, -128), 127);
+            rs += c;
+            packed[j >> 2] |= (uint32_t)(c & 0xFF) << (8 * (j & 3));
+        }
+        reinterpret_cast<uint2*>(q)[v] = make_uint2(packed[0], packed[1]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
+    rowsum_out = rs;
+    s_out = s;
+}
+
+// Dynamic shared memory: (blockDim.x / 32) * 4 * max K bytes (row + gain per warp).
+template <int CAP>
+__global__ void __launch_bounds__(256) quant_warp_kernel(const __grid_constant__ QuantBatch<CAP> b,
+                                                         int kmax) {
+    extern __shared__ __align__(16) uint4 xs_all[];
+    pdl_launch_dependents();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5;
+    const int row = blockIdx.x * (blockDim.x >> 5) + warp;  // (problem, token) index
+    if (row >= b.count * b.M) return;
+    const int p = row / b.M, m = row % b.M;
+    const QuantProblem& pr = b.p[p];
+    float s;
+    int rs;
+    uint4* xs = xs_all + (size_t)warp * (kmax >> 2);
+    quantize_row_warp(pr.x + (int64_t)m * pr.K, pr.gain, b.eps, pr.K, pr.q + (int64_t)m * pr.K, xs,
+                      xs + (kmax >> 3), s, rs);
+    if ((threadIdx.x & 31) == 0) {
         pr.s_x[m] = s;
         if (pr.rowsum) pr.rowsum[m] = rs;
     }
