@@ -38,7 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "BitLinear W1.58A8 tokens/s; % roofline (GEMV HBM GB/s, GEMM int8 TOPS)"
-DECODE_KERNEL_SOURCES = ("common.cuh", "quant.cuh", "decode.cuh")
+DECODE_KERNEL_SOURCES = ("common.cuh", "decode.cuh")
 FALLBACK_HBM_GBS = 6650.0
 
 

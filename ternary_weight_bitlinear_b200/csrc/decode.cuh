@@ -18,10 +18,13 @@
 //    waits on the kernel before it (programmatic dependent launch), so weight
 //    traffic overlaps the activation quantisation that precedes it.
 //  * Unpacking never materialises ternary values: bit pair i of a packed byte
-//    is selected in place with the mask 3 << 2i, so each 32-bit word gives four
+//    is selected in place with the mask 3 << 2i, so each 32-bit word gives
 //    u8 operands code_i << 2i (code = t+1) for dp4a against four int8 codes.
-//    The factor 4^i is shifted out exactly at the end and t = code - 1 is
-//    folded in with the row sum of the codes: sum q*t = sum q*code - sum q.
+//    Only bit pairs 0-2 are masked: the whole byte is sum_i 4^i code_i, so
+//    dp4a of the unmasked word accumulates sum_i 4^i S_i and 4^3 S_3 is that
+//    total minus the three masked sums (exact integer arithmetic).  The
+//    factor 4^i is shifted out at the end and t = code - 1 is folded in with
+//    the row sum of the codes: sum q*t = sum q*code - sum q.
 //  * After the wait, each CTA stages the int8 codes, scales and row sums of the
 //    problems its rows belong to in shared memory (they are reused by every
 //    row of a problem); batches too large to stage read them from L2.
@@ -32,7 +35,6 @@
 #pragma once
 
 #include "common.cuh"
-#include "quant.cuh"
 
 namespace bl {
 
@@ -115,6 +117,7 @@ struct Walker {
     int r_end;  // first row of p outside the range
     int c;      // chunk of the row
     int K;
+    int max_rows;  // whole rows per copy for this problem (1 when rows are chunked)
     const uint8_t* P;
 
     __device__ __forceinline__ void enter(const DecBatch<CAP>& b, int np, int64_t r0, int64_t hi) {
@@ -123,6 +126,7 @@ struct Walker {
         if (p >= b.count) return;
         const DecProblem& pr = b.p[p];
         K = pr.K;
+        max_rows = K <= kDecChunk ? min(kDecMaxRows, kDecChunk / K) : 1;
         P = pr.P;
         const int64_t lim = hi - pr.byte0;  // rows with first byte < hi
         r_end = (int)(lim <= 0 ? 0 : min((lim + K - 1) / K, pr.R));
@@ -143,7 +147,7 @@ struct Walker {
     __device__ __forceinline__ bool valid(const DecBatch<CAP>& b) const { return p < b.count; }
     // whole rows in the next copy (short rows are copied two at a time)
     __device__ __forceinline__ int rows() const {
-        return K <= kDecChunk ? min(min(kDecMaxRows, kDecChunk / K), r_end - r) : 1;
+        return min(max_rows, r_end - r);
     }
     __device__ __forceinline__ int bytes() const {
         return K <= kDecChunk ? rows() * K : min(kDecChunk, K - c * kDecChunk);
@@ -174,7 +178,9 @@ __device__ __forceinline__ RingSpot ring_spot(uint32_t off, int bytes) {
     return {wrap ? 0u : off, (wrap ? (uint32_t)kDecRing - off : 0u) + (uint32_t)bytes};
 }
 
-// acc[i] += sum over the 16 bytes of (bit pair i of w, left in place) * q
+// acc[i] += sum over the 16 bytes of (bit pair i of w, left in place) * q for
+// i < 3; acc[3] += sum of (whole byte) * q.  finish_acc() turns acc[3] into
+// the bit-pair-3 sum once the row is complete.
 __device__ __forceinline__ void dot16(const uint4 w4, const uint4 q4, int (&acc)[4]) {
     const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
     const uint32_t q[4] = {q4.x, q4.y, q4.z, q4.w};
@@ -183,24 +189,49 @@ __device__ __forceinline__ void dot16(const uint4 w4, const uint4 q4, int (&acc)
         acc[0] = dp4a_us(w[j] & 0x03030303u, q[j], acc[0]);
         acc[1] = dp4a_us(w[j] & 0x0C0C0C0Cu, q[j], acc[1]);
         acc[2] = dp4a_us(w[j] & 0x30303030u, q[j], acc[2]);
-        acc[3] = dp4a_us(w[j] & 0xC0C0C0C0u, q[j], acc[3]);
+        acc[3] = dp4a_us(w[j], q[j], acc[3]);
     }
 }
 
-__device__ __forceinline__ void store_output(const DecProblem& pr, int64_t idx, int acc, float s_x) {
-    if (pr.epi == kEpiI32) {
-        static_cast<int32_t*>(pr.y)[idx] = acc;
+// whole-byte sum minus the bit-pair-0..2 sums = 4^3 * (bit-pair-3 sum).  Every
+// partial stays below 2^31 in magnitude: a byte is at most 0xAA (codes <= 2),
+// 170 * 128 * 65536 < 2^31.
+__device__ __forceinline__ void finish_acc(int (&acc)[4]) {
+    acc[3] -= acc[0] + acc[1] + acc[2];
+}
+
+// The output constants of the problem being consumed, kept in registers.
+struct EpiConsts {
+    void* y;
+    const uint16_t* residual;
+    int64_t N;
+    int64_t R;
+    float beta;
+    int epi;
+    __device__ __forceinline__ void load(const DecProblem& pr) {
+        y = pr.y;
+        residual = pr.residual;
+        N = pr.N;
+        R = pr.R;
+        beta = pr.beta;
+        epi = pr.epi;
+    }
+};
+
+__device__ __forceinline__ void store_output(const EpiConsts& e, int64_t idx, int acc, float s_x) {
+    if (e.epi == kEpiI32) {
+        static_cast<int32_t*>(e.y)[idx] = acc;
         return;
     }
-    const float y = __fdiv_rn(__fmul_rn(__int2float_rn(acc), pr.beta), s_x);
-    if (pr.epi == kEpiF32) {
-        static_cast<float*>(pr.y)[idx] = y;
+    const float y = __fdiv_rn(__fmul_rn(__int2float_rn(acc), e.beta), s_x);
+    if (e.epi == kEpiF32) {
+        static_cast<float*>(e.y)[idx] = y;
     } else {
         uint16_t b = float_to_bf16_bits(y);
-        if (pr.residual)
+        if (e.residual)
             b = float_to_bf16_bits(
-                __fadd_rn(bf16_bits_to_float(__ldcg(pr.residual + idx)), bf16_bits_to_float(b)));
-        static_cast<uint16_t*>(pr.y)[idx] = b;
+                __fadd_rn(bf16_bits_to_float(__ldcg(e.residual + idx)), bf16_bits_to_float(b)));
+        static_cast<uint16_t*>(e.y)[idx] = b;
     }
 }
 
@@ -334,14 +365,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
     const int8_t* qbase = nullptr;
     float sx[MT];
     int rsum[MT];
+    EpiConsts ec{};
+    int qoff_cur = 0;
     while (done < issued) {  // refill() keeps the queue non-empty until the walk ends
         const ItemDesc d = my_descs[done % kDecSlots];
-        if (d.p != cur_p) {  // entering a problem: cache its activation data
+        if (d.p != cur_p) {  // entering a problem: cache its activation and output data
             cur_p = d.p;
             const DecProblem& pr = b.p[cur_p];
             K = pr.K;
+            ec.load(pr);
             if (staged) {
-                qbase = qs + qoff[cur_p - pa];
+                qoff_cur = qoff[cur_p - pa];
+                qbase = qs + qoff_cur;
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     sx[m] = sxs[(cur_p - pa) * kDecMaxTokens + m];
@@ -366,18 +401,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         const uint8_t* wbase = ring + d.at;
         const int8_t* qrow = qbase + d.c * kDecChunk;
+        // the staged codes addressed from the shared array itself, so that the
+        // compiler emits shared-memory loads with 32-bit addresses
+        const int8_t* qrow_s = qs + qoff_cur + d.c * kDecChunk;
         if (d.rows == 2) {
             // two rows: half-warp h takes row d.r + h
             const int h = lane >> 4, hl = lane & 15;
             const uint4* wp = reinterpret_cast<const uint4*>(wbase + h * K);
             const int nvec = K >> 4;
             if (staged) {
-#pragma unroll 4
+#pragma unroll 2
                 for (int v = hl; v < nvec; v += 16) {
                     const uint4 w4 = wp[v];
 #pragma unroll
                     for (int m = 0; m < MT; ++m)
-                        dot16(w4, reinterpret_cast<const uint4*>(qrow + m * K)[v], acc[m]);
+                        dot16(w4, reinterpret_cast<const uint4*>(qrow_s + m * K)[v], acc[m]);
                 }
             } else {
                 for (int v = hl; v < nvec; v += 16) {
@@ -392,12 +430,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
             const uint4* wp = reinterpret_cast<const uint4*>(wbase);
             const int nvec = d.bytes >> 4;
             if (staged) {
-#pragma unroll 4
+#pragma unroll 2
                 for (int v = lane; v < nvec; v += 32) {
                     const uint4 w4 = wp[v];
 #pragma unroll
                     for (int m = 0; m < MT; ++m)
-                        dot16(w4, reinterpret_cast<const uint4*>(qrow + m * K)[v], acc[m]);
+                        dot16(w4, reinterpret_cast<const uint4*>(qrow_s + m * K)[v], acc[m]);
                 }
             } else {
                 for (int v = lane; v < nvec; v += 32) {
@@ -414,26 +452,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
         ++done;
         refill();
         if ((d.c + 1) * kDecChunk >= K || d.rows == 2) {  // the item ends its row(s)
-            const DecProblem& pr = b.p[cur_p];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) finish_acc(acc[m]);
             if (d.rows == 2) {
+                const int i = (lane >> 2) & 3;
+                const int64_t o = (int64_t)i * ec.R + d.r + (lane >> 4);
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     const int tot = half_reduce4(acc[m], lane);
-                    if ((lane & 3) == 0) {
-                        const int i = (lane >> 2) & 3;
-                        store_output(pr, (int64_t)m * pr.N + (int64_t)i * pr.R + d.r + (lane >> 4),
-                                     (tot >> (2 * i)) - rsum[m], sx[m]);
-                    }
+                    if ((lane & 3) == 0)
+                        store_output(ec, m * ec.N + o, (tot >> (2 * i)) - rsum[m], sx[m]);
                 }
             } else {
+                const int i = lane >> 3;
+                const int64_t o = (int64_t)i * ec.R + d.r;
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     const int tot = warp_reduce4(acc[m], lane);
-                    if ((lane & 7) == 0) {
-                        const int i = lane >> 3;
-                        store_output(pr, (int64_t)m * pr.N + (int64_t)i * pr.R + d.r,
-                                     (tot >> (2 * i)) - rsum[m], sx[m]);
-                    }
+                    if ((lane & 7) == 0)
+                        store_output(ec, m * ec.N + o, (tot >> (2 * i)) - rsum[m], sx[m]);
                 }
             }
         }

@@ -12,11 +12,11 @@
 //   warp 0      TMA producer: per stage, the 128x128-byte int8 activation tile
 //               (A operand, 128-byte swizzle, rows past M zero-filled) and the
 //               64x128-byte packed weight tile; no multicast.
-//   warps 1-4   expansion: 2-bit codes -> int8 codes written straight into the
+//   warps 1-8   expansion: 2-bit codes -> int8 codes written straight into the
 //               128-byte-swizzled K-major B operand (256 rows) in shared memory.
-//   warp 5      one thread issues tcgen05.mma.cta_group::1.kind::i8
+//   warp 9      one thread issues tcgen05.mma.cta_group::1.kind::i8
 //               (M=128, N=256, K=32) into a TMEM accumulator (2 buffers).
-//   warps 6-9   epilogue: each thread owns one token (a TMEM lane of its
+//   warps 10-13 epilogue: each thread owns one token (a TMEM lane of its
 //               warp's quadrant) and 256 output rows: tcgen05.ld, minus the
 //               token's row sum, rescale, 16-byte stores of contiguous outputs.
 // Loads run up to kTcStages stages ahead; expanded operands are double-buffered.
@@ -36,8 +36,10 @@ constexpr int kTcBK = 128;        // K bytes per stage (one 128-byte swizzle ato
 constexpr int kTcPackRows = 64;   // packed rows per tile (x 4 bit pairs = kTcBN)
 constexpr int kTcStages = 5;      // load stages (A + packed weights)
 constexpr int kTcExp = 2;         // expanded-B buffers
-constexpr int kTcThreads = 320;
-constexpr int kTcEpiWarp0 = 6;
+constexpr int kTcExpWarps = 8;    // expansion warps (1 .. 8)
+constexpr int kTcMmaWarp = 1 + kTcExpWarps;
+constexpr int kTcEpiWarp0 = kTcMmaWarp + 1;
+constexpr int kTcThreads = 32 * (kTcEpiWarp0 + 4);
 constexpr int kTcABytes = kTcBM * kTcBK;          // 16 KB activations
 constexpr int kTcBBytes = kTcBN * kTcBK;          // 32 KB expanded codes
 constexpr int kTcPBytes = kTcPackRows * kTcBK;    // 8 KB packed codes
@@ -51,6 +53,7 @@ constexpr int kTcOffTmem = kTcOffBar + 8 * kTcNumBars;
 constexpr int kTcSmemBytes = kTcOffTmem + 16 + 1024;   // + alignment slack
 constexpr uint32_t kTcTmemCols = 2 * kTcBN;           // two accumulators
 static_assert(kTcSmemBytes <= 227 * 1024, "shared memory budget");
+static_assert((kTcPackRows * 8) % (32 * kTcExpWarps) == 0, "expansion items per thread");
 
 struct TcArgs {
     const uint8_t* P;          // [R,K] (through tmap_p)
@@ -245,7 +248,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
             mbar_init(empty_bar(s), 1);
         }
         for (int e = 0; e < kTcExp; ++e) {
-            mbar_init(bready_bar(e), 4);
+            mbar_init(bready_bar(e), kTcExpWarps);
             mbar_init(bfree_bar(e), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -255,7 +258,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
         mbar_init(mma_done_bar, 1);
         mbar_init_fence();
     }
-    if (warp == 5) tmem_alloc(smem_addr(tmem_slot), kTcTmemCols);
+    if (warp == kTcMmaWarp) tmem_alloc(smem_addr(tmem_slot), kTcTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -289,9 +292,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
                 for (uint32_t j = inflight_from; j < g; ++j)
                     mbar_wait(full_bar((int)(j % kTcStages)), (j / kTcStages) & 1u);
         }
-    } else if (warp >= 1 && warp <= 4) {
+    } else if (warp >= 1 && warp <= kTcExpWarps) {
         // ---------------- expansion: 2-bit codes -> int8 B tile ----------------
-        const int e0 = threadIdx.x - 32;  // 0..127
+        const int e0 = threadIdx.x - 32;  // 0 .. 32*kTcExpWarps-1
         uint32_t g = 0;
         for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
             for (int ks = 0; ks < kstages; ++ks, ++g) {
@@ -302,8 +305,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
                 const uint8_t* pk = sm + kTcOffP + s * kTcPBytes;
                 uint8_t* bt = sm + kTcOffB + e * kTcBBytes;
 #pragma unroll
-                for (int it = 0; it < 4; ++it) {
-                    const int item = e0 + it * 128;  // (packed row, 16-byte chunk)
+                for (int it = 0; it < kTcPackRows * 8 / (32 * kTcExpWarps); ++it) {
+                    const int item = e0 + it * 32 * kTcExpWarps;  // (packed row, 16-byte chunk)
                     const int rr = item >> 3, ch = item & 7;
                     const uint4 w = *reinterpret_cast<const uint4*>(pk + rr * kTcBK + ch * 16);
 #pragma unroll
@@ -321,7 +324,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
                 if (lane == 0) mbar_arrive(bready_bar(e));
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kTcMmaWarp) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             uint32_t g = 0, tl = 0;
@@ -386,7 +389,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kTcMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTcTmemCols);
     }
