@@ -138,6 +138,101 @@ __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ---- correctly rounded division by a reused divisor ---------------------------
+// RN(a / s) for a divisor s > 0 shared by many quotients (a token's scale).
+// With y = RN(1/s) computed once, q = RN(a*y) is refined by one FMA step
+// (Markstein's correction, q + (a - q*s)*y), which leaves q a faithful
+// rounding of a/s.  The remainder a - q*s of a faithful quotient is exactly
+// representable, so one more FMA gives it exactly, and q = RN(a/s) holds iff
+// |a - q*s| < ulp(q)*s/2: the floats next to q are one ulp(q) away when q is
+// not a power of two, and a/s is never a midpoint (it would need more than
+// 24 significant bits times s to equal a).  Where that check cannot vouch for
+// q -- a zero, tiny, huge or non-finite operand, q a power of two, or the
+// bound failing -- the quotient comes from __fdiv_rn instead.
+struct RecipDiv {
+    float s;
+    float y;
+};
+
+__device__ __forceinline__ RecipDiv recip_div_init(float s) { return {s, __frcp_rn(s)}; }
+
+__device__ __forceinline__ float recip_div(float a, const RecipDiv& d) {
+    float q = __fmul_rn(a, d.y);
+    q = __fmaf_rn(__fmaf_rn(-q, d.s, a), d.y, q);
+    const float r = __fmaf_rn(-q, d.s, a);
+    const uint32_t qb = __float_as_uint(q);
+    const uint32_t e = (qb >> 23) & 0xFFu;                  // biased exponent of q
+    const float half_ulp = __uint_as_float((e - 24u) << 23);  // ulp(q)/2 = 2^(e-151)
+    const float h = __fmul_rn(half_ulp, d.s);               // exact when normal
+    const uint32_t ab = __float_as_uint(a) & 0x7FFFFFFFu;
+    const bool ok = ab >= 0x0D800000u && ab <= 0x71800000u &&  // 2^-100 <= |a| <= 2^100
+                    e >= 25u && e <= 253u && (qb & 0x007FFFFFu) != 0u &&
+                    __float_as_uint(h) >= 0x00800000u && fabsf(r) < h;
+    if (ok) return q;
+    return __fdiv_rn(a, d.s);
+}
+
+// The rescale y = RN32(RN32(acc * beta) / s) for many outputs sharing a
+// token's divisor s.  Same method as recip_div, split so that the common case
+// has no branch: when beta and s both lie in [2^-40, 2^40] and
+// 1 <= |acc| <= 2^31, a = RN(acc*beta) lies in [2^-40, 2^71] and q in
+// [2^-80, 2^111], so every intermediate is a normal float and only the
+// rounding test itself (and q a power of two) is left per output; acc = 0
+// gives a = q = +0 exactly (beta > 0).  Outputs whose test fails, or any
+// divisor or beta outside the range, go through scale_slow.
+struct PairDiv {
+    float s;
+    float y;   // RN(1/s)
+    float ns;  // -s
+    bool fast;
+};
+
+__device__ __forceinline__ PairDiv pair_div_init(float s, float beta) {
+    const bool fast = s >= 0x1p-40f && s <= 0x1p40f && beta >= 0x1p-40f && beta <= 0x1p40f;
+    return {s, __frcp_rn(s), -s, fast};
+}
+
+// Candidate quotient; ok is set when it is proven to be RN(a/s).
+__device__ __forceinline__ float scale_fast(int acc, float beta, const PairDiv& d, bool& ok) {
+    const float a = __fmul_rn(__int2float_rn(acc), beta);
+    float q = __fmul_rn(a, d.y);
+    q = __fmaf_rn(__fmaf_rn(q, d.ns, a), d.y, q);
+    const float r = __fmaf_rn(q, d.ns, a);  // exact remainder of the faithful q
+    const uint32_t qb = __float_as_uint(q);
+    // ulp(q)/2 * s, exact: a power of two times s, normal in this range
+    const float h = __fmul_rn(__uint_as_float((qb & 0x7F800000u) - 0x0C000000u), d.s);
+    ok = acc == 0 || ((qb & 0x007FFFFFu) != 0u && fabsf(r) < h);
+    return q;
+}
+
+__device__ __noinline__ float scale_slow(int acc, float beta, float s, float y) {
+    return recip_div(__fmul_rn(__int2float_rn(acc), beta), RecipDiv{s, y});
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// y[j] = RN32(RN32((v[j] - rsum) * beta) / s) for 16 outputs.
+__device__ __forceinline__ void scale16(const uint32_t* v, int rsum, float beta, const PairDiv& d,
+                                        float (&y)[16]) {
+    uint32_t bad = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        bool ok;
+        y[j] = scale_fast((int)v[j] - rsum, beta, d, ok);
+        bad |= (ok ? 0u : 1u) << j;
+    }
+    if (!d.fast) bad = 0xFFFFu;
+    if (bad) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (bad & (1u << j)) y[j] = scale_slow((int)v[j] - rsum, beta, d.s, d.y);
+    }
+}
+
 // ---- integer dot products ----------------------------------------------------
 // d = c + sum_{j<4} a.u8[j] * b.s8[j]
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {

@@ -218,12 +218,13 @@ struct EpiConsts {
     }
 };
 
-__device__ __forceinline__ void store_output(const EpiConsts& e, int64_t idx, int acc, float s_x) {
+__device__ __forceinline__ void store_output(const EpiConsts& e, int64_t idx, int acc,
+                                             const RecipDiv& s_x) {
     if (e.epi == kEpiI32) {
         static_cast<int32_t*>(e.y)[idx] = acc;
         return;
     }
-    const float y = __fdiv_rn(__fmul_rn(__int2float_rn(acc), e.beta), s_x);
+    const float y = recip_div(__fmul_rn(__int2float_rn(acc), e.beta), s_x);
     if (e.epi == kEpiF32) {
         static_cast<float*>(e.y)[idx] = y;
     } else {
@@ -363,7 +364,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
     int acc[MT][4];
     int cur_p = -1, K = 0;
     const int8_t* qbase = nullptr;
-    float sx[MT];
+    RecipDiv sx[MT];
     int rsum[MT];
     EpiConsts ec{};
     int qoff_cur = 0;
@@ -379,14 +380,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
                 qbase = qs + qoff_cur;
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
-                    sx[m] = sxs[(cur_p - pa) * kDecMaxTokens + m];
+                    sx[m] = recip_div_init(sxs[(cur_p - pa) * kDecMaxTokens + m]);
                     rsum[m] = rss[(cur_p - pa) * kDecMaxTokens + m];
                 }
             } else {
                 qbase = pr.q;
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
-                    sx[m] = pr.epi == kEpiI32 ? 1.0f : __ldcg(pr.s_x + m);
+                    sx[m] = recip_div_init(pr.epi == kEpiI32 ? 1.0f : __ldcg(pr.s_x + m));
                     rsum[m] = __ldcg(pr.rowsum + m);
                 }
             }

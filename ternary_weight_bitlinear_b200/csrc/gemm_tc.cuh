@@ -16,9 +16,11 @@
 //               128-byte-swizzled K-major B operand (256 rows) in shared memory.
 //   warp 9      one thread issues tcgen05.mma.cta_group::1.kind::i8
 //               (M=128, N=256, K=32) into a TMEM accumulator (2 buffers).
-//   warps 10-13 epilogue: each thread owns one token (a TMEM lane of its
-//               warp's quadrant) and 256 output rows: tcgen05.ld, minus the
-//               token's row sum, rescale, 16-byte stores of contiguous outputs.
+//   warps 10-17 epilogue: each thread owns one token (a TMEM lane of its
+//               warp's quadrant) and half of the 256 output rows: tcgen05.ld,
+//               minus the token's row sum, rescale (division by the token's
+//               scale through its reciprocal, exactness checked per output),
+//               16-byte stores of contiguous outputs.
 // Loads run up to kTcStages stages ahead; expanded operands are double-buffered.
 // Every mbarrier wait is bounded (records BL_ERR_TIMEOUT and unwinds).
 #pragma once
@@ -39,7 +41,8 @@ constexpr int kTcExp = 2;         // expanded-B buffers
 constexpr int kTcExpWarps = 8;    // expansion warps (1 .. 8)
 constexpr int kTcMmaWarp = 1 + kTcExpWarps;
 constexpr int kTcEpiWarp0 = kTcMmaWarp + 1;
-constexpr int kTcThreads = 32 * (kTcEpiWarp0 + 4);
+constexpr int kTcEpiWarps = 8;    // two per TMEM lane quadrant, each half the columns
+constexpr int kTcThreads = 32 * (kTcEpiWarp0 + kTcEpiWarps);
 constexpr int kTcABytes = kTcBM * kTcBK;          // 16 KB activations
 constexpr int kTcBBytes = kTcBN * kTcBK;          // 32 KB expanded codes
 constexpr int kTcPBytes = kTcPackRows * kTcBK;    // 8 KB packed codes
@@ -54,6 +57,7 @@ constexpr int kTcSmemBytes = kTcOffTmem + 16 + 1024;   // + alignment slack
 constexpr uint32_t kTcTmemCols = 2 * kTcBN;           // two accumulators
 static_assert(kTcSmemBytes <= 227 * 1024, "shared memory budget");
 static_assert((kTcPackRows * 8) % (32 * kTcExpWarps) == 0, "expansion items per thread");
+static_assert(kTcEpiWarps == 8 && (kTcEpiWarp0 + kTcEpiWarps) * 32 <= 1024, "epilogue warps");
 
 struct TcArgs {
     const uint8_t* P;          // [R,K] (through tmap_p)
@@ -152,22 +156,24 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk16) {
     return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((chunk16 ^ (row & 7)) << 4));
 }
 
-// Store 32 consecutive outputs y[m, n0 .. n0+31] of one token (scalar path:
-// only rows < R, i.e. n0 + j with j < valid).
-__device__ __forceinline__ float tc_scale(int acc, float beta, float s_x) {
-    return __fdiv_rn(__fmul_rn(__int2float_rn(acc), beta), s_x);
+// y = RN32(RN32(acc * beta) / s_x)
+__device__ __forceinline__ float tc_scale(int acc, float beta, const PairDiv& s_x) {
+    return recip_div(__fmul_rn(__int2float_rn(acc), beta), RecipDiv{s_x.s, s_x.y});
 }
 
+// Store 32 consecutive outputs y[m, n0 .. n0+31] of one token (scalar path:
+// only rows < R, i.e. n0 + j with j < valid).
 __device__ __forceinline__ void tc_store_row32(const TcArgs& a, int64_t base, const uint32_t (&v)[32], int rsum,
-                               float s_x, int valid) {
+                               const PairDiv& s_x, int valid) {
     if (a.vec_ok && valid == 32) {
         if (a.epi == kEpiBF16) {
             uint32_t w[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                uint32_t lo = float_to_bf16_bits(tc_scale((int)v[2 * j] - rsum, a.beta, s_x));
-                uint32_t hi = float_to_bf16_bits(tc_scale((int)v[2 * j + 1] - rsum, a.beta, s_x));
-                w[j] = lo | (hi << 16);
+            for (int g = 0; g < 2; ++g) {
+                float y[16];
+                scale16(v + 16 * g, rsum, a.beta, s_x, y);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) w[8 * g + j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
             }
             if (a.residual) {
                 const uint4* rp = reinterpret_cast<const uint4*>(a.residual + base);
@@ -178,29 +184,32 @@ __device__ __forceinline__ void tc_store_row32(const TcArgs& a, int64_t base, co
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
                         const uint32_t x = w[4 * c + h];
-                        const uint32_t lo = float_to_bf16_bits(__fadd_rn(
-                            bf16_bits_to_float(rr[h] & 0xFFFFu), bf16_bits_to_float(x & 0xFFFFu)));
-                        const uint32_t hi = float_to_bf16_bits(__fadd_rn(
-                            bf16_bits_to_float(rr[h] >> 16), bf16_bits_to_float(x >> 16)));
-                        w[4 * c + h] = lo | (hi << 16);
+                        w[4 * c + h] = pack_bf16x2(
+                            __fadd_rn(bf16_bits_to_float(rr[h] & 0xFFFFu), bf16_bits_to_float(x & 0xFFFFu)),
+                            __fadd_rn(bf16_bits_to_float(rr[h] >> 16), bf16_bits_to_float(x >> 16)));
                     }
                 }
             }
             uint4* yp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.y) + base);
 #pragma unroll
             for (int c = 0; c < 4; ++c) yp[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        } else if (a.epi == kEpiF32) {
+            uint4* yp = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.y) + base);
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                float y[16];
+                scale16(v + 16 * g, rsum, a.beta, s_x, y);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    yp[4 * g + c] = make_uint4(__float_as_uint(y[4 * c]), __float_as_uint(y[4 * c + 1]),
+                                               __float_as_uint(y[4 * c + 2]), __float_as_uint(y[4 * c + 3]));
+            }
         } else {
             uint4* yp = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.y) + base);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t w[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int acc = (int)v[4 * c + h] - rsum;
-                    w[h] = a.epi == kEpiI32 ? (uint32_t)acc : __float_as_uint(tc_scale(acc, a.beta, s_x));
-                }
-                yp[c] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+            for (int c = 0; c < 8; ++c)
+                yp[c] = make_uint4(v[4 * c] - rsum, v[4 * c + 1] - rsum, v[4 * c + 2] - rsum,
+                                   v[4 * c + 3] - rsum);
         }
         return;
     }
@@ -253,7 +262,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(accfull_bar(b), 1);
-            mbar_init(accempty_bar(b), 4);
+            mbar_init(accempty_bar(b), kTcEpiWarps);
         }
         mbar_init(mma_done_bar, 1);
         mbar_init_fence();
@@ -359,20 +368,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
     } else {
         // ---------------- epilogue: one token per thread ----------------
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const int half = (warp - kTcEpiWarp0) >> 2;  // which 128 of the 256 columns
         uint32_t tl = 0;
         for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tl) {
             const int tn = (int)(t / a.tiles_m), tm = (int)(t % a.tiles_m);
             const int buf = (int)(tl & 1);
             const int m = tm * kTcBM + q * 32 + lane;  // this thread's token
             const bool live = m < a.M;
-            const float sx = (live && a.epi != kEpiI32) ? __ldcg(a.s_x + m) : 1.0f;
+            const PairDiv sx = pair_div_init((live && a.epi != kEpiI32) ? __ldcg(a.s_x + m) : 1.0f, a.beta);
             const int rsum = live ? __ldcg(a.rowsum + m) : 0;
             const bool got = mbar_wait(accfull_bar(buf), (tl >> 1) & 1u);
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kTcBN);
 #pragma unroll 1
-            for (int c0 = 0; c0 < kTcBN; c0 += 32) {
+            for (int c0 = half * (kTcBN / 2); c0 < (half + 1) * (kTcBN / 2); c0 += 32) {
                 uint32_t v[32];
                 tmem_ld32(taddr + (uint32_t)c0, v);
                 const int i = c0 / kTcPackRows;                       // bit pair
