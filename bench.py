@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-skinny", action="store_true",
+                    help="skip the batched-decode (8/32/64 tokens) measurements")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the M=4096 prefill measurement reported beside the headline")
     return ap.parse_args()
@@ -182,7 +184,7 @@ class DecodeWorkload:
             if key not in gains:
                 gains[key] = torch.from_numpy(c["gain"].view(np.int16)).view(torch.bfloat16).to(dev)
             self.problems.append(dict(
-                layer=l, x=self.x_dev[xo:xo + M * p.K].view(M, p.K), P=P, beta=float(beta.item()),
+                layer=l, name=p.name, x=self.x_dev[xo:xo + M * p.K].view(M, p.K), P=P, beta=float(beta.item()),
                 gain=gains[key], y=self.y_dev[yo:yo + M * p.N].view(M, p.N), K=p.K, N=p.N))
             self.weight_bytes += P.numel()
             xo += M * p.K
@@ -314,6 +316,64 @@ class PrefillWorkload:
         out["frac_of_int8_peak"] = out["gemm_tops"] / peak
         out["tokens_per_s"] = self.M / (tot_fwd_ms / 1000.0)  # one pass over the 5 projections
         return out
+
+
+class SkinnyWorkload:
+    """Batched decode (5..64 tokens): every projection of all decoder layers
+    with its own M-token input (per-token scales drawn from U(0.1, 10), no
+    RMSNorm, bf16 out), over the packed weights of a DecodeWorkload.  Times the
+    weight-streaming GEMV on already-quantised codes (its HBM roofline) and the
+    whole batched forward (quantise + GEMV)."""
+
+    def __init__(self, dec, M):
+        import ternary_weight_bitlinear_b200 as B
+        WL = dec.WL
+        self.B, self.M = B, M
+        items, qitems = [], []
+        self.gemv_bytes = 0
+        for q in dec.problems:
+            c = WL.config3_projection(q["layer"], q["name"], M)
+            x = torch.from_numpy(c["x"].view(np.int16)).view(torch.bfloat16).cuda()
+            y = torch.empty((M, q["N"]), dtype=torch.bfloat16, device="cuda")
+            items.append(dict(x=x, P=q["P"], beta=q["beta"], y=y))
+            qq, sx, rs = B.bitlinear_act_quant(x)
+            qitems.append(dict(q=qq, s_x=sx, rowsum=rs, P=q["P"], beta=q["beta"], y=y))
+            self.gemv_bytes += q["P"].numel() + M * q["K"] + 2 * M * q["N"] + 8 * M
+        self.items, self.qitems = items, qitems
+        self.batch = B.make_batch(items)
+        self.qbatch = B.make_quantized_batch(qitems)
+        self.ws = torch.empty(B.bitlinear_forward_batch_workspace_size(self.batch, M),
+                              dtype=torch.uint8, device="cuda")
+        self.qws = torch.empty(max(16, B.bitlinear_quantized_batch_workspace_size(M)),
+                               dtype=torch.uint8, device="cuda")
+        self.graphs = {}
+        for mode in ("gemv", "forward"):
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                self.run(mode)
+            torch.cuda.current_stream().wait_stream(s)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.run(mode)
+            torch.cuda.synchronize()
+            self.graphs[mode] = g
+
+    def run(self, mode):
+        if mode == "gemv":
+            self.B.bitlinear_forward_quantized_batch(self.qbatch, self.M, workspace=self.qws)
+        else:
+            self.B.bitlinear_forward_batch(self.batch, self.M, 0.0, workspace=self.ws)
+
+    def measure(self, reps, warmup, world, hbm):
+        ms_g = timed(self.graphs["gemv"].replay, reps, warmup, world) / reps
+        ms_f = timed(self.graphs["forward"].replay, reps, warmup, world) / reps
+        gbs = self.gemv_bytes / (ms_g / 1000.0) / 1e9
+        return {"M": self.M, "gemv_us": ms_g * 1000.0, "gemv_gbs": gbs, "frac_of_hbm": gbs / hbm,
+                "forward_us": ms_f * 1000.0, "tokens_per_s": world * self.M / (ms_f / 1000.0),
+                "launches_per_step": {"gemv": (len(self.items) + 63) // 64,
+                                      "forward": 1 + (len(self.items) + 63) // 64}}
 
 
 def measured_int8_peak():
@@ -518,6 +578,18 @@ def main():
     ms_e2e = max_over_ranks(timed(e2e_step, args.steps, args.warmup, world), world)
     e2e_value = world * wl.M * args.steps / (ms_e2e / 1000.0)
 
+    hbm, hbm_src = measured_peaks()
+    skinny = None
+    if not args.no_skinny:
+        skinny = {"workload": "batched decode: M tokens through the 210 projections of 30 "
+                              "BitNet-2B4T layers (independent inputs, per-token scales "
+                              "U(0.1, 10)), no RMSNorm, bf16 out; weights of the headline",
+                  "by_M": {}}
+        for Ms in (8, 32, 64):
+            sw = SkinnyWorkload(wl, Ms)
+            skinny["by_M"][str(Ms)] = sw.measure(max(3, min(args.steps, 20)), max(args.warmup, 2),
+                                                 world, hbm)
+            del sw
     prefill = None
     if not args.no_prefill:
         pw = PrefillWorkload()
@@ -527,7 +599,6 @@ def main():
     if status != 0:
         raise RuntimeError("device status %d after the timed region" % status)
 
-    hbm, hbm_src = measured_peaks()
     gemv_launch_ms = ms_gemv / args.steps
     bytes_per_launch = wl.gemv_bytes
     achieved = bytes_per_launch / (gemv_launch_ms / 1000.0) / 1e9
@@ -546,6 +617,7 @@ def main():
                              "launch_us": gemv_launch_ms * 1000.0,
                              "bytes_per_launch": bytes_per_launch},
                 "variants": variants,
+                "skinny": skinny,
                 "prefill": prefill,
                 "e2e": {"value": e2e_value, "unit": "tokens/s",
                         "h2d_bytes_per_step": wl.h2d_bytes, "d2h_bytes_per_step": wl.d2h_bytes},

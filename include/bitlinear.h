@@ -185,12 +185,25 @@ typedef struct {
     bl_out_dtype y_dtype;
 } bl_quantized_problem;
 
+/* Workspace that lets bitlinear_forward_quantized_batch split row tiles between
+ * CTAs for 5 <= M <= 64 (0 for other M): one flag and one block of int32
+ * partial sums per CTA. */
+bl_status bitlinear_quantized_batch_workspace_size(int64_t M, size_t* bytes);
+
 /* `count` (1..BL_MAX_BATCH) independent bitlinear_forward_quantized problems
  * with the same M.  Problems may share q (projections of one input, e.g. the
  * q|k|v or gate|up projections of a decoder layer).  For M <= 4 one launch
- * streams every problem's weights once.  No workspace. */
+ * streams every problem's weights once; for 5 <= M <= 64 one launch per 64
+ * problems does (tensor cores, weights expanded into tensor memory).
+ *   workspace  device or NULL.  With at least
+ *          bitlinear_quantized_batch_workspace_size(M) bytes every CTA streams
+ *          an equal share of the weights; without it (NULL or smaller) shares
+ *          are cut at 128-row tile boundaries, with the same results.  A
+ *          workspace serves one call at a time; its contents need no
+ *          initialisation and are left for the next call. */
 bl_status bitlinear_forward_quantized_batch(const bl_quantized_problem* problems, int count,
-                                            int64_t M, void* stream);
+                                            int64_t M, void* workspace, size_t workspace_bytes,
+                                            void* stream);
 
 /* Matmul and rescale on activations already quantised by bitlinear_act_quant
  * (so several projections can share one quantisation):

@@ -42,7 +42,8 @@ SIGNATURES = {
     "bitlinear_device_status": ([_P], _INT),
     "bitlinear_forward_batch_workspace_size": ([_P, _INT, _I64, ctypes.POINTER(_SZ)], _INT),
     "bitlinear_forward_batch": ([_P, _INT, _I64, _F32, _P, _SZ, _P], _INT),
-    "bitlinear_forward_quantized_batch": ([_P, _INT, _I64, _P], _INT),
+    "bitlinear_quantized_batch_workspace_size": ([_I64, ctypes.POINTER(_SZ)], _INT),
+    "bitlinear_forward_quantized_batch": ([_P, _INT, _I64, _P, _SZ, _P], _INT),
 }
 
 
@@ -253,9 +254,20 @@ def make_quantized_batch(items):
     return arr
 
 
-def bitlinear_forward_quantized_batch(batch, M, stream=None):
+def bitlinear_quantized_batch_workspace_size(M):
+    n = ctypes.c_size_t()
+    _check("bitlinear_quantized_batch_workspace_size",
+           lib().bitlinear_quantized_batch_workspace_size(M, ctypes.byref(n)))
+    return n.value
+
+
+def bitlinear_forward_quantized_batch(batch, M, workspace=None, stream=None):
+    """``workspace``: None, or a uint8 CUDA tensor of at least
+    bitlinear_quantized_batch_workspace_size(M) bytes (equal CTA shares for
+    5 <= M <= 64)."""
     _check("bitlinear_forward_quantized_batch", lib().bitlinear_forward_quantized_batch(
-        ctypes.cast(batch, _P), len(batch), M, _stream(stream)))
+        ctypes.cast(batch, _P), len(batch), M, _ptr(workspace),
+        0 if workspace is None else workspace.numel(), _stream(stream)))
 
 
 def bitlinear_forward_quantized(q, s_x, rowsum, P, beta, out_dtype=torch.bfloat16, residual=None,

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <climits>
 #include <cstdio>
 #include <map>
@@ -18,6 +20,7 @@
 #include "glue.cuh"
 #include "pack.cuh"
 #include "quant.cuh"
+#include "skinny.cuh"
 
 namespace {
 
@@ -143,6 +146,16 @@ struct WsSlices {
     float* s_x;
     int32_t* rowsum;
 };
+
+// Tail of a forward workspace used by the 5..64-token kernel when a row tile
+// is shared by several CTAs: one flag and one block of int32 partial sums
+// (npad x 128) per CTA.
+bool skinny_m(int64_t M) { return M >= kSkMinTokens && M <= kSkMaxTokens; }
+int64_t sk_npad(int64_t M) { return (M + 15) / 16 * 16; }
+int64_t sk_flag_bytes() { return round_up(8 * kSkMaxGrid, 256); }
+int64_t sk_ws_bytes(int64_t M) {
+    return skinny_m(M) ? sk_flag_bytes() + (int64_t)kSkMaxGrid * sk_npad(M) * 128 * 4 : 0;
+}
 
 WsSlices ws_slices(char* w, int64_t M, int64_t K) {
     return {reinterpret_cast<int8_t*>(w), reinterpret_cast<float*>(w + ws_q_bytes(M, K)),
@@ -339,15 +352,86 @@ bl_status run_gemm(const int8_t* q, const float* s_x, const int32_t* rowsum, con
                   stream, map_q, map_p, a);
 }
 
+// A launch epoch for the partial-sum flags: never 0 (a cleared flag), and
+// distinct between launches of one process.
+unsigned long long next_epoch() {
+    static std::atomic<unsigned long long> e{
+        0x9E3779B97F4A7C15ull ^
+        (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count()};
+    unsigned long long v;
+    do { v = e.fetch_add(1); } while (v == 0);
+    return v;
+}
+
+// 5..64 tokens: the weight-streaming tensor-core kernel over up to kSkCap
+// problems per launch.  With a workspace of sk_ws_bytes(M) the CTA shares are
+// exactly equal (row tiles may be split); without one they are cut at row-tile
+// boundaries.
+bl_status run_skinny(const DecodeJob* jobs, int count, int64_t M, void* ws, size_t ws_bytes, int dev,
+                     const DeviceInfo& info, cudaStream_t stream) {
+    if (prepare_kernel(reinterpret_cast<const void*>(skinny_tc_kernel), dev, info, kSkThreads,
+                       kSkSmemBytes) < 0)
+        return BL_ERR_CUDA;
+    static thread_local SkBatch b;  // ~22 KB: kept off the stack
+    const int npad = (int)sk_npad(M);
+    const bool split = ws && ws_bytes >= (size_t)sk_ws_bytes(M);
+    for (int c0 = 0; c0 < count; c0 += kSkCap) {
+        const int n = std::min(kSkCap, count - c0);
+        b = SkBatch{};
+        b.count = n;
+        b.M = (int)M;
+        b.npad = npad;
+        int64_t items = 0;
+        for (int i = 0; i < n; ++i) {
+            const DecodeJob& j = jobs[c0 + i];
+            SkProblem& p = b.p[i];
+            p.s_x = j.s_x;
+            p.rowsum = j.rowsum;
+            p.y = j.y;
+            p.residual = j.residual;
+            p.N = j.N;
+            p.R = (int)(j.N / 4);
+            p.K = (int)j.K;
+            p.tiles = (p.R + kSkRows - 1) / kSkRows;
+            p.kst = (p.K + kSkItemK - 1) / kSkItemK;
+            p.beta = j.beta;
+            p.epi = j.epi;
+            p.item0 = items;
+            items += (int64_t)p.tiles * p.kst;
+            if (!make_map_u8(&b.tmap_p[i], j.P, (uint64_t)j.K, (uint64_t)p.R, kSkBK, kSkRows,
+                             CU_TENSOR_MAP_SWIZZLE_128B) ||
+                !make_map_u8(&b.tmap_q[i], j.q, (uint64_t)j.K, (uint64_t)M, kSkBK, (uint32_t)npad,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+                return BL_ERR_CUDA;
+        }
+        b.total = items;
+        b.split = split ? 1 : 0;
+        if (split) {
+            b.flags = static_cast<unsigned long long*>(ws);
+            b.part = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + sk_flag_bytes());
+        }
+        b.epoch = next_epoch();
+        const int64_t grid = std::max<int64_t>(
+            1, std::min<int64_t>(items, std::min<int64_t>(info.sms, kSkMaxGrid)));
+        bl_status st = launch(skinny_tc_kernel, dim3((unsigned)grid), dim3(kSkThreads),
+                              (size_t)kSkSmemBytes, stream, b);
+        if (st != BL_OK) return st;
+    }
+    return BL_OK;
+}
+
 // Matmul + epilogue on pre-quantised activations, any M: the decode kernel
-// for up to four tokens, the tensor-core GEMM beyond.
+// for up to four tokens, the weight-streaming tensor-core kernel for 5..64,
+// the tensor-core GEMM beyond.  sk_ws: the optional split workspace of the
+// 5..64-token kernel.
 bl_status run_quantized(const int8_t* q, const float* s_x, const int32_t* rowsum, const uint8_t* P,
                         float beta, int64_t M, int64_t K, int64_t N, void* y, int epi,
                         const uint16_t* residual, int dev, const DeviceInfo& info,
-                        cudaStream_t stream) {
-    if (M > kDecMaxTokens)
-        return run_gemm(q, s_x, rowsum, P, beta, M, K, N, y, epi, residual, dev, info, stream);
+                        cudaStream_t stream, void* sk_ws = nullptr, size_t sk_ws_len = 0) {
     DecodeJob j = {q, s_x, rowsum, P, y, residual, K, N, beta, epi};
+    if (M > kSkMaxTokens)
+        return run_gemm(q, s_x, rowsum, P, beta, M, K, N, y, epi, residual, dev, info, stream);
+    if (M > kDecMaxTokens) return run_skinny(&j, 1, M, sk_ws, sk_ws_len, dev, info, stream);
     return run_decode(&j, 1, (int)M, dev, info, stream);
 }
 
@@ -479,7 +563,7 @@ bl_status bitlinear_forward_workspace_size(int64_t M, int64_t K, int64_t N, size
     if (!bytes) return BL_ERR_NULL;
     bl_status st = check_shape(M, K, N);
     if (st != BL_OK) return st;
-    *bytes = M == 0 ? 0 : (size_t)ws_problem_bytes(M, K);
+    *bytes = M == 0 ? 0 : (size_t)(ws_problem_bytes(M, K) + sk_ws_bytes(M));
     return BL_OK;
 }
 
@@ -495,7 +579,8 @@ bl_status bitlinear_forward(const uint16_t* x, const uint16_t* gain, float eps, 
     if (!x || !P || !y) return BL_ERR_NULL;
     if (!aligned16(x) || !aligned16(P) || !aligned16(y) || (gain && !aligned16(gain)))
         return BL_ERR_ALIGN;
-    if (!workspace || workspace_bytes < (size_t)ws_problem_bytes(M, K)) return BL_ERR_WORKSPACE;
+    const int64_t own = ws_problem_bytes(M, K);
+    if (!workspace || workspace_bytes < (size_t)(own + sk_ws_bytes(M))) return BL_ERR_WORKSPACE;
     if (!aligned16(workspace)) return BL_ERR_ALIGN;
     int dev;
     DeviceInfo info;
@@ -505,7 +590,8 @@ bl_status bitlinear_forward(const uint16_t* x, const uint16_t* gain, float eps, 
     const WsSlices w = ws_slices(static_cast<char*>(workspace), M, K);
     QuantProblem qp = {x, gain, w.q, w.s_x, w.rowsum, (int)K};
     if ((st = run_quant(&qp, 1, M, eps, dev, info, s)) != BL_OK) return st;
-    return run_quantized(w.q, w.s_x, w.rowsum, P, beta, M, K, N, y, epi, nullptr, dev, info, s);
+    return run_quantized(w.q, w.s_x, w.rowsum, P, beta, M, K, N, y, epi, nullptr, dev, info, s,
+                         static_cast<char*>(workspace) + own, (size_t)sk_ws_bytes(M));
 }
 
 bl_status bitlinear_forward_batch_workspace_size(const bl_problem* probs, int count, int64_t M,
@@ -518,6 +604,7 @@ bl_status bitlinear_forward_batch_workspace_size(const bl_problem* probs, int co
         if (st != BL_OK) return st;
         total += M == 0 ? 0 : ws_problem_bytes(M, probs[i].K);
     }
+    total += sk_ws_bytes(M);
     *bytes = (size_t)total;
     return BL_OK;
 }
@@ -558,6 +645,7 @@ bl_status bitlinear_forward_batch(const bl_problem* probs, int count, int64_t M,
     }
     if ((st = run_quant(qp, count, M, eps, dev, info, s)) != BL_OK) return st;
     if (M <= kDecMaxTokens) return run_decode(jobs, count, (int)M, dev, info, s);
+    if (skinny_m(M)) return run_skinny(jobs, count, M, w, (size_t)sk_ws_bytes(M), dev, info, s);
     for (int i = 0; i < count; ++i) {
         const DecodeJob& j = jobs[i];
         st = run_quantized(j.q, j.s_x, j.rowsum, j.P, j.beta, M, j.K, j.N, j.y, j.epi, j.residual,
@@ -586,8 +674,16 @@ bl_status bitlinear_forward_quantized(const int8_t* q, const float* s_x, const i
                          static_cast<cudaStream_t>(stream));
 }
 
+bl_status bitlinear_quantized_batch_workspace_size(int64_t M, size_t* bytes) {
+    if (!bytes) return BL_ERR_NULL;
+    if (M < 0) return BL_ERR_SHAPE;
+    *bytes = (size_t)sk_ws_bytes(M);
+    return BL_OK;
+}
+
 bl_status bitlinear_forward_quantized_batch(const bl_quantized_problem* probs, int count,
-                                            int64_t M, void* stream) {
+                                            int64_t M, void* workspace, size_t workspace_bytes,
+                                            void* stream) {
     if (!probs) return BL_ERR_NULL;
     if (count < 1 || count > BL_MAX_BATCH || M < 0) return BL_ERR_SHAPE;
     DecodeJob jobs[BL_MAX_BATCH];
@@ -611,6 +707,10 @@ bl_status bitlinear_forward_quantized_batch(const bl_quantized_problem* probs, i
     if ((st = current_device(&dev, &info)) != BL_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (M <= kDecMaxTokens) return run_decode(jobs, count, (int)M, dev, info, s);
+    if (skinny_m(M)) {
+        if (workspace && !aligned16(workspace)) return BL_ERR_ALIGN;
+        return run_skinny(jobs, count, M, workspace, workspace_bytes, dev, info, s);
+    }
     for (int i = 0; i < count; ++i) {
         const DecodeJob& j = jobs[i];
         st = run_quantized(j.q, j.s_x, j.rowsum, j.P, j.beta, M, j.K, j.N, j.y, j.epi, j.residual,

@@ -54,6 +54,25 @@ def test_workspace_sizes(L):
         B.bitlinear_forward_workspace_size(1, 2561, 16)
 
 
+def test_skinny_workspace_sizes(L):
+    """5..64 tokens add one split area (a flag and npad x 128 int32 per CTA)."""
+    Q = B.bitlinear_quantized_batch_workspace_size
+    assert Q(0) == Q(1) == Q(4) == Q(65) == Q(4096) == 0
+    s5, s16, s17, s64 = Q(5), Q(16), Q(17), Q(64)
+    assert 0 < s5 == s16 < s17 < s64           # npad 16, 16, 32, 64
+    assert s64 - s16 == 3 * (s17 - s16)        # linear in npad
+    assert s64 >= 148 * 64 * 128 * 4          # room for every CTA of a B200
+    own = 8 * 2560 + 2 * 256                  # codes + s_x + row sums (256-byte slices)
+    assert B.bitlinear_forward_workspace_size(8, 2560, 640) == own + Q(8)
+    assert B.bitlinear_forward_workspace_size(4, 2560, 640) == 4 * 2560 + 2 * 256
+    sz = ctypes.c_size_t()
+    arr = _batch(7, K=2560, N=640)
+    assert L.bitlinear_forward_batch_workspace_size(arr, 7, 8, ctypes.byref(sz)) == 0
+    assert sz.value == 7 * own + Q(8)          # one split area for the whole batch
+    assert L.bitlinear_quantized_batch_workspace_size(8, None) == 1
+    assert L.bitlinear_quantized_batch_workspace_size(-1, ctypes.byref(sz)) == 2
+
+
 def _fwd(L, x=P16, gain=NULL, P=P16, M=1, K=256, N=128, y=P16, dt=0, ws=P16, wsb=1 << 30):
     return L.bitlinear_forward(x, gain, 1e-5, P, 1.0, M, K, N, y, dt, ws, wsb, NULL)
 
