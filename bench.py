@@ -62,15 +62,21 @@ def parse_args():
 # ---------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------
-def dist_setup():
+def dist_setup(timeout_s=300):
+    """One process per GPU under torchrun (NCCL); the same plumbing runs on
+    CPU-only hosts over gloo (tests)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group(
-            "nccl", timeout=datetime.timedelta(seconds=300),
-            device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group(
+                "nccl", timeout=datetime.timedelta(seconds=timeout_s),
+                device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group(
+                "gloo", timeout=datetime.timedelta(seconds=timeout_s))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -82,11 +88,19 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """The slowest rank's value (every rank calls this, in the same order)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank, world, ms):
+    """Whole-job units per second: every rank processed units_per_rank in at
+    most ms (the max over ranks of the device-timed region)."""
+    return world * units_per_rank / (ms / 1000.0)
 
 
 # ---------------------------------------------------------------------------
@@ -557,7 +571,7 @@ def main():
         ms = timed(head.replay, args.steps, args.warmup, world)
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
-    value = world * wl.M * args.steps / (ms / 1000.0)
+    value = job_throughput(wl.M * args.steps, world, ms)
 
     # the GEMV kernel alone on the same batch (pre-quantised codes): its roofline
     ms_gemv = max_over_ranks(timed(wl.graphs["gemv_token"].replay, args.steps, args.warmup, world),
@@ -565,7 +579,7 @@ def main():
     variants = {}
     for mode in ("layer_batch", "per_call", "gemv_only"):
         t = max_over_ranks(timed(wl.graphs[mode].replay, args.steps, args.warmup, world), world)
-        variants[mode] = {"tokens_per_s": world * wl.M * args.steps / (t / 1000.0),
+        variants[mode] = {"tokens_per_s": job_throughput(wl.M * args.steps, world, t),
                           "ms_per_step": t / args.steps, "launches_per_step": wl.launches[mode]}
     variants["gemv_only"]["note"] = ("the layer_batch GEMV launches alone (17.4 MB each): "
                                      "bound by per-launch ramp, see profiles/")
@@ -576,7 +590,7 @@ def main():
         head.replay()
         wl.y_host.copy_(wl.y_dev, non_blocking=True)
     ms_e2e = max_over_ranks(timed(e2e_step, args.steps, args.warmup, world), world)
-    e2e_value = world * wl.M * args.steps / (ms_e2e / 1000.0)
+    e2e_value = job_throughput(wl.M * args.steps, world, ms_e2e)
 
     hbm, hbm_src = measured_peaks()
     skinny = None

@@ -266,6 +266,15 @@ bl_status bitlinear_relu2_mul(const uint16_t* a, const uint16_t* b, int64_t n, u
  * bounded wait since the last call. */
 bl_status bitlinear_device_status(void* stream);
 
+/* Failure-detection self-test (diagnostics; the pages have no counterpart).
+ * Launches one CTA that waits on a shared-memory barrier nothing arrives on,
+ * with a wait limit of limit_ns (clamped to 1 us .. 10 s) instead of the
+ * kernels' 2 s: the wait runs out, records the timeout in the device status
+ * word and the kernel returns, as every bounded wait of the library does.  The
+ * next bitlinear_device_status() returns BL_ERR_TIMEOUT and clears the word;
+ * the context stays usable.  Asynchronous on `stream`. */
+bl_status bitlinear_selftest_wait_timeout(int64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -40,6 +40,7 @@ SIGNATURES = {
     "bitlinear_relu2_mul": ([_P, _P, _I64, _P, _P], _INT),
     "bitlinear_forward_noalloc": ([_P, _P, _F32, _P, _F32, _I64, _I64, _I64, _P, _INT, _P], _INT),
     "bitlinear_device_status": ([_P], _INT),
+    "bitlinear_selftest_wait_timeout": ([_I64, _P], _INT),
     "bitlinear_forward_batch_workspace_size": ([_P, _INT, _I64, ctypes.POINTER(_SZ)], _INT),
     "bitlinear_forward_batch": ([_P, _INT, _I64, _F32, _P, _SZ, _P], _INT),
     "bitlinear_quantized_batch_workspace_size": ([_I64, ctypes.POINTER(_SZ)], _INT),
@@ -301,6 +302,12 @@ def bitlinear_relu2_mul(a, b, out=None, stream=None):
     _check("bitlinear_relu2_mul", lib().bitlinear_relu2_mul(_ptr(a), _ptr(b), a.numel(), _ptr(z),
                                                             _stream(stream)))
     return z
+
+
+def bitlinear_selftest_wait_timeout(limit_ns, stream=None):
+    """Launch the bounded-wait self-test (see include/bitlinear.h)."""
+    _check("bitlinear_selftest_wait_timeout",
+           lib().bitlinear_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 def bitlinear_device_status(stream=None):

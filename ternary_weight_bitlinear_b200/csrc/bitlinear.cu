@@ -769,6 +769,16 @@ bl_status bitlinear_device_status(void* stream) {
     return (v & kStatusTimeout) ? BL_ERR_TIMEOUT : BL_OK;
 }
 
+bl_status bitlinear_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+    int dev;
+    DeviceInfo info;
+    bl_status st;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    const unsigned long long lim =
+        (unsigned long long)std::min<int64_t>(std::max<int64_t>(limit_ns, 1000), 10000000000ll);
+    return launch(wait_selftest_kernel, dim3(1), dim3(32), 0, static_cast<cudaStream_t>(stream), lim);
+}
+
 bl_status bitlinear_forward_noalloc(const uint16_t* x, const uint16_t* gain, float eps,
                                     const uint8_t* P, float beta, int64_t M, int64_t K,
                                     int64_t N, void* y, bl_out_dtype y_dtype, void* stream) {
