@@ -29,6 +29,8 @@ using namespace bl;
 constexpr int kQuantThreads = 256;
 constexpr int kSmallBatch = 8;  // parameter-table size of small batches
 constexpr int64_t kQuantWarpMinRows = 1024;  // rows from which a warp per row pays off
+constexpr int kQuantRegVpt1 = 10;  // 16-byte vectors per thread, one warp per row: K <= 2560
+constexpr int kQuantRegVpt4 = 7;   // ... four warps per row: K <= 7168
 
 // ---- device properties and per-kernel launch settings ---------------------
 struct DeviceInfo {
@@ -175,7 +177,22 @@ bl_status launch_quant_cap(const QuantProblem* probs, int count, int64_t M, floa
         b.p[i] = probs[i];
         kmax = std::max(kmax, probs[i].K);
     }
-    if (kmax <= kQuantWarpMaxK && (int64_t)count * M >= kQuantWarpMinRows) {
+    const int64_t rows = (int64_t)count * M;
+    if (rows >= kQuantWarpMinRows && kmax <= 32 * 8 * kQuantRegVpt1) {
+        // many rows (prefill), short rows: one warp per row, held in registers
+        auto fn = quant_reg_kernel<1, kQuantRegVpt1, CAP>;
+        if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, 128, 0) < 0)
+            return BL_ERR_CUDA;
+        return launch(fn, dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, stream, b);
+    }
+    if (rows >= kQuantWarpMinRows && kmax <= 128 * 8 * kQuantRegVpt4) {
+        // many rows, longer rows: four warps per row, held in registers
+        auto fn = quant_reg_kernel<4, kQuantRegVpt4, CAP>;
+        if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, 128, 0) < 0)
+            return BL_ERR_CUDA;
+        return launch(fn, dim3((unsigned)rows), dim3(128), 0, stream, b);
+    }
+    if (kmax <= kQuantWarpMaxK && rows >= kQuantWarpMinRows) {
         // many rows (prefill): one warp per row, up to 8 rows per CTA; few rows
         // (decode) go to one CTA per row below, which has the lower latency
         const int wpb = (int)std::max<int64_t>(1, std::min<int64_t>(8, 65536 / (4 * (int64_t)kmax)));
@@ -183,7 +200,6 @@ bl_status launch_quant_cap(const QuantProblem* probs, int count, int64_t M, floa
         const int64_t smem = (int64_t)wpb * 4 * kmax;
         if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, 32 * wpb, smem) < 0)
             return BL_ERR_CUDA;
-        const int64_t rows = (int64_t)count * M;
         return launch(fn, dim3((unsigned)((rows + wpb - 1) / wpb)), dim3(32 * wpb), (size_t)smem,
                       stream, b, kmax);
     }

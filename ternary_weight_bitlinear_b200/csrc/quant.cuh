@@ -381,4 +381,164 @@ __global__ void __launch_bounds__(256) quant_warp_kernel(const __grid_constant__
     }
 }
 
+// ---- rows held in registers: W warps per row, up to VPT vectors per thread ----
+// Same arithmetic as quantize_row.  Every 16-byte load of the row is issued
+// before any use, so a thread has VPT loads in flight; nothing is staged in
+// shared memory.  W = 1: one warp per row (4 rows per CTA, no block barriers);
+// W = 4: one CTA per row (K up to 128 * 8 * VPT).
+template <int W, int VPT, int CAP>
+__global__ void __launch_bounds__(128, 4) quant_reg_kernel(const __grid_constant__ QuantBatch<CAP> b) {
+    static_assert(W == 1 || W == 4, "one warp or one CTA per row");
+    constexpr int RPC = 4 / W;  // rows per CTA
+    constexpr int NTR = 32 * W; // threads per row
+    __shared__ double red_hi[4], red_lo[4];
+    __shared__ float red_f[4];
+    __shared__ int red_i[4];
+    pdl_launch_dependents();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = warp % W;
+    const int row = blockIdx.x * RPC + warp / W;
+    if (row >= b.count * b.M) return;  // uniform over a row's warps; W = 4: over the CTA
+    const int p = row / b.M, m = row % b.M;
+    const QuantProblem pr = b.p[p];
+    const int t = sub * 32 + lane;
+    const int nvec = pr.K >> 3;
+    const uint4* xv = reinterpret_cast<const uint4*>(pr.x + (int64_t)m * pr.K);
+    const uint4* gv = reinterpret_cast<const uint4*>(pr.gain);
+    const bool norm = pr.gain != nullptr;
+
+    uint4 xr[VPT];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int v = t + i * NTR;
+        xr[i] = v < nvec ? __ldcg(xv + v) : make_uint4(0u, 0u, 0u, 0u);  // zeros add nothing
+    }
+
+    // sum over the row's threads, in a fixed order (W = 4: warps in index order)
+    auto row_sum_dd = [&](double hi, double lo) -> double {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const double ohi = __shfl_down_sync(0xffffffffu, hi, o);
+            const double olo = __shfl_down_sync(0xffffffffu, lo, o);
+            if (lane < o) dd_merge(hi, lo, ohi, olo);
+        }
+        if (W == 1) {
+            hi = __shfl_sync(0xffffffffu, hi, 0);
+            lo = __shfl_sync(0xffffffffu, lo, 0);
+            return __dadd_rn(hi, lo);
+        }
+        if (lane == 0) { red_hi[warp] = hi; red_lo[warp] = lo; }
+        __syncthreads();
+        double h = red_hi[0], l = red_lo[0];
+        for (int w = 1; w < W; ++w) dd_merge(h, l, red_hi[w], red_lo[w]);
+        __syncthreads();
+        return __dadd_rn(h, l);
+    };
+    auto row_max = [&](float v) -> float {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (W == 1) return v;
+        if (lane == 0) red_f[warp] = v;
+        __syncthreads();
+        float r = red_f[0];
+        for (int w = 1; w < W; ++w) r = fmaxf(r, red_f[w]);
+        return r;  // the next barrier (in row_sum_int) orders the reuse of red_f
+    };
+    auto row_sum_int = [&](int v) -> int {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (W == 1) return v;
+        if (lane == 0) red_i[warp] = v;
+        __syncthreads();
+        int r = 0;
+        for (int w = 0; w < W; ++w) r += red_i[w];
+        return r;
+    };
+
+    float r = 1.0f, mx = 0.0f;
+    if (norm) {
+        double ss0 = 0.0, ss1 = 0.0;  // plain binary64 sums of the exact squares
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            float f[8];
+            unpack8_bf16(xr[i], f);
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                ss0 = __fma_rn((double)f[j], (double)f[j], ss0);
+                ss1 = __fma_rn((double)f[j + 1], (double)f[j + 1], ss1);
+            }
+        }
+        const double approx = row_sum_dd(__dadd_rn(ss0, ss1), 0.0);
+        if (!rms_factor_bounded(approx, pr.K, b.eps, r)) {
+            // rare: the interval straddles a rounding boundary; take the sum
+            // exactly (re-reading the row from L2 keeps this path's registers
+            // away from the common one)
+            double hi = 0.0, lo = 0.0;
+#pragma unroll 1
+            for (int v = t; v < nvec; v += NTR) {
+                float f[8];
+                unpack8_bf16(__ldcg(xv + v), f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const double d = (double)f[j];
+                    dd_add(hi, lo, __dmul_rn(d, d));  // exact square of a bf16 value
+                }
+            }
+            r = rms_factor(row_sum_dd(hi, lo), pr.K, b.eps);
+        }
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int v = t + i * NTR;
+            if (v < nvec) {
+                float f[8], g[8];
+                unpack8_bf16(xr[i], f);
+                unpack8_bf16(__ldg(gv + v), g);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(norm_elem(f[j], r, g[j])));
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            float f[8];
+            unpack8_bf16(xr[i], f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(f[j]));
+        }
+    }
+    const float s = __fdiv_rn(127.0f, fmaxf(row_max(mx), kScaleFloor));
+
+    int rs = 0;
+    int8_t* q = pr.q + (int64_t)m * pr.K;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int v = t + i * NTR;
+        if (v < nvec) {
+            float f[8];
+            unpack8_bf16(xr[i], f);
+            if (norm) {
+                float g[8];
+                unpack8_bf16(__ldg(gv + v), g);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] = norm_elem(f[j], r, g[j]);
+            }
+            uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                int c = __float2int_rn(__fmul_rn(f[j], s));  // round half to even
+                c = min(max(c, -128), 127);
+                rs += c;
+                packed[j >> 2] |= (uint32_t)(c & 0xFF) << (8 * (j & 3));
+            }
+            reinterpret_cast<uint2*>(q)[v] = make_uint2(packed[0], packed[1]);
+        }
+    }
+    rs = row_sum_int(rs);
+    if (t == 0) {
+        pr.s_x[m] = s;
+        if (pr.rowsum) pr.rowsum[m] = rs;
+    }
+}
+
 }  // namespace bl

@@ -99,7 +99,12 @@ def special_rows(x):
 
 
 @pytest.mark.parametrize("norm", [False, True])
-@pytest.mark.parametrize("M,K", [(1, 16), (3, 256), (4, 2560), (7, 6912), (64, 2560), (257, 272)])
+@pytest.mark.parametrize("M,K", [(1, 16), (3, 256), (4, 2560), (7, 6912), (64, 2560), (257, 272),
+                                 # 1024+ rows: the register-resident kernels (one warp per
+                                 # row up to K = 2560, four up to 7168) and, past that, the
+                                 # shared-memory warp kernel
+                                 (1024, 2560), (1031, 6912), (1100, 272), (1024, 2576),
+                                 (1025, 7168), (1024, 8192)])
 def test_act_quant_matches_oracle(M, K, norm):
     x = special_rows(WL.activations(M, K, seed=M * 131 + K, outlier_frac=0.001))
     gain = WL.gain(K, seed=K) if norm else None
