@@ -390,6 +390,81 @@ class SkinnyWorkload:
                                       "forward": 1 + (len(self.items) + 63) // 64}}
 
 
+class FfnChainWorkload:
+    """Config 5: M=16 tokens through the FFN blocks of all 30 layers in order
+    (RMSNorm -> gate, up -> relu(gate)^2 * up -> sub-norm -> down -> + residual),
+    the packed gate/up/down weights of the headline workload.  Each layer is
+    act_quant, one batched gate|up GEMV, relu2_mul, act_quant and the down
+    GEMV with the residual epilogue: 5 launches per layer, captured in one
+    graph that also restores the input."""
+
+    def __init__(self, dec, M=16):
+        import ternary_weight_bitlinear_b200 as B
+        WL = dec.WL
+        self.B, self.WL, self.M = B, WL, M
+        byname = {(q["layer"], q["name"]): q for q in dec.problems}
+        self.x0 = torch.from_numpy(WL.config5_input(M).view(np.int16)).view(torch.bfloat16).cuda()
+        self.x = self.x0.clone()
+        H, I = WL.HIDDEN, WL.INTERMEDIATE
+        self.layers = []
+        self.weight_bytes = 0
+        for l in range(dec.layers):
+            g, u, d = byname[(l, "gate")], byname[(l, "up")], byname[(l, "down")]
+            gi = torch.from_numpy(WL.gain(H, 1000 * (l + 1) + 10).view(np.int16)).view(torch.bfloat16).cuda()
+            gs = torch.from_numpy(WL.gain(I, 1000 * (l + 1) + 11).view(np.int16)).view(torch.bfloat16).cuda()
+            self.layers.append(dict(g=g, u=u, d=d, gi=gi, gs=gs))
+            self.weight_bytes += g["P"].numel() + u["P"].numel() + d["P"].numel()
+        dev = "cuda"
+        self.q1 = torch.empty((M, H), dtype=torch.int8, device=dev)
+        self.s1 = torch.empty(M, dtype=torch.float32, device=dev)
+        self.r1 = torch.empty(M, dtype=torch.int32, device=dev)
+        self.a = torch.empty((M, I), dtype=torch.bfloat16, device=dev)
+        self.b = torch.empty((M, I), dtype=torch.bfloat16, device=dev)
+        self.z = torch.empty((M, I), dtype=torch.bfloat16, device=dev)
+        self.q2 = torch.empty((M, I), dtype=torch.int8, device=dev)
+        self.s2 = torch.empty(M, dtype=torch.float32, device=dev)
+        self.r2 = torch.empty(M, dtype=torch.int32, device=dev)
+        self.ws = torch.empty(max(16, B.bitlinear_quantized_batch_workspace_size(M)),
+                              dtype=torch.uint8, device=dev)
+        for L in self.layers:
+            L["gu"] = B.make_quantized_batch([
+                dict(q=self.q1, s_x=self.s1, rowsum=self.r1, P=L["g"]["P"], beta=L["g"]["beta"], y=self.a),
+                dict(q=self.q1, s_x=self.s1, rowsum=self.r1, P=L["u"]["P"], beta=L["u"]["beta"], y=self.b)])
+            L["dn"] = B.make_quantized_batch([
+                dict(q=self.q2, s_x=self.s2, rowsum=self.r2, P=L["d"]["P"], beta=L["d"]["beta"],
+                     y=self.x, residual=self.x)])
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.run()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.run()
+        torch.cuda.synchronize()
+
+    def run(self):
+        B, eps, M = self.B, self.WL.RMS_EPS, self.M
+        self.x.copy_(self.x0)
+        for L in self.layers:
+            B.bitlinear_act_quant(self.x, L["gi"], eps, q=self.q1, s_x=self.s1, rowsum=self.r1)
+            B.bitlinear_forward_quantized_batch(L["gu"], M, workspace=self.ws)
+            B.bitlinear_relu2_mul(self.a, self.b, out=self.z)
+            B.bitlinear_act_quant(self.z, L["gs"], eps, q=self.q2, s_x=self.s2, rowsum=self.r2)
+            B.bitlinear_forward_quantized_batch(L["dn"], M, workspace=self.ws)
+
+    def measure(self, reps, warmup, world, hbm):
+        ms = timed(self.graph.replay, reps, warmup, world) / reps
+        gbs = self.weight_bytes / (ms / 1000.0) / 1e9
+        return {"workload": "config 5: M=%d tokens through the FFN blocks of %d BitNet-2B4T "
+                            "layers in order (RMSNorm, gate|up, relu2*, sub-norm, down, "
+                            "+residual); attention omitted" % (self.M, len(self.layers)),
+                "chain_us": ms * 1000.0, "tokens_per_s": job_throughput(self.M, world, ms),
+                "packed_weight_gbs": gbs, "frac_of_hbm": gbs / hbm,
+                "launches_per_step": 5 * len(self.layers)}
+
+
 def measured_int8_peak():
     """Dense int8 tensor peak: the measured bf16 GEMM burst x the nominal 2x ratio."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -604,6 +679,11 @@ def main():
             skinny["by_M"][str(Ms)] = sw.measure(max(3, min(args.steps, 20)), max(args.warmup, 2),
                                                  world, hbm)
             del sw
+    ffn = None
+    if not args.no_skinny:
+        fw = FfnChainWorkload(wl)
+        ffn = fw.measure(max(3, min(args.steps, 20)), max(args.warmup, 2), world, hbm)
+        del fw
     prefill = None
     if not args.no_prefill:
         pw = PrefillWorkload()
@@ -632,6 +712,7 @@ def main():
                              "bytes_per_launch": bytes_per_launch},
                 "variants": variants,
                 "skinny": skinny,
+                "ffn_chain": ffn,
                 "prefill": prefill,
                 "e2e": {"value": e2e_value, "unit": "tokens/s",
                         "h2d_bytes_per_step": wl.h2d_bytes, "d2h_bytes_per_step": wl.d2h_bytes},

@@ -84,26 +84,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     }
 }
 
-// Self-test of the bounded waits: thread 0 waits on a barrier nothing arrives
-// on until limit_ns pass, then records the timeout and returns.
-__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
-    __shared__ __align__(8) uint64_t bar;
-    if (threadIdx.x == 0) {
-        mbar_init(smem_addr(&bar), 1);
-        mbar_init_fence();
-    }
-    __syncthreads();
-    if (threadIdx.x != 0) return;
-    const unsigned long long t0 = globaltimer_ns();
-    for (uint32_t n = 0;; ++n) {
-        if (mbar_try_wait(smem_addr(&bar), 0)) return;
-        if ((n & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) {
-            atomicOr(&g_status, kStatusTimeout);
-            return;
-        }
-    }
-}
-
 // ---- bulk copies (TMA engine, no multicast) ---------------------------------
 // Global -> this CTA's shared memory; completion counted in bytes on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16.

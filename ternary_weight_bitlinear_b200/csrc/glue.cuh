@@ -1,4 +1,5 @@
-// glue.cuh -- elementwise FFN glue between BitLinear projections.
+// glue.cuh -- elementwise FFN glue between BitLinear projections, and the
+// self-test kernel of the bounded waits.
 //
 // "BitNet" transformers model doc, model details: the FFN uses squared ReLU
 // (hidden_act "relu2") in a gated form, z = relu(gate)^2 * up, computed here
@@ -39,6 +40,26 @@ __global__ void __launch_bounds__(kGlueThreads) relu2_mul_kernel(const uint16_t*
         *reinterpret_cast<uint4*>(z + base) = make_uint4(o[0], o[1], o[2], o[3]);
     } else {
         for (int64_t i = base; i < n; ++i) z[i] = relu2_mul_one(__ldcg(a + i), __ldcg(b + i));
+    }
+}
+
+// Self-test of the bounded waits: thread 0 waits on a barrier nothing arrives
+// on until limit_ns pass, then records the timeout and returns.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar), 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    if (threadIdx.x != 0) return;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t n = 0;; ++n) {
+        if (mbar_try_wait(smem_addr(&bar), 0)) return;
+        if ((n & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+            atomicOr(&g_status, kStatusTimeout);
+            return;
+        }
     }
 }
 
