@@ -215,24 +215,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
-// y[j] = RN32(RN32((v[j] - rsum) * beta) / s) for 16 outputs.
-__device__ __forceinline__ void scale16(const uint32_t* v, int rsum, float beta, const PairDiv& d,
-                                        float (&y)[16]) {
-    uint32_t bad = 0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        bool ok;
-        y[j] = scale_fast((int)v[j] - rsum, beta, d, ok);
-        bad |= (ok ? 0u : 1u) << j;
-    }
-    if (!d.fast) bad = 0xFFFFu;
-    if (bad) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if (bad & (1u << j)) y[j] = scale_slow((int)v[j] - rsum, beta, d.s, d.y);
-    }
-}
-
 // ---- integer dot products ----------------------------------------------------
 // d = c + sum_{j<4} a.u8[j] * b.s8[j]
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {

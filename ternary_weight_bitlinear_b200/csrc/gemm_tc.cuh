@@ -156,6 +156,49 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk16) {
     return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((chunk16 ^ (row & 7)) << 4));
 }
 
+// scale_fast for two outputs at once on the paired fp32 pipe (f32x2).
+__device__ __forceinline__ void scale_fast2(int a0, int a1, float beta, const PairDiv& d, float& y0,
+                                            float& y1, bool& ok0, bool& ok1) {
+    float r0, r1;
+    asm("{\n\t.reg .b64 A, Q, R, B, Y, N;\n\t"
+        "mov.b64 A, {%4, %5};\n\t"
+        "mov.b64 B, {%6, %6};\n\t"
+        "mov.b64 Y, {%7, %7};\n\t"
+        "mov.b64 N, {%8, %8};\n\t"
+        "mul.rn.f32x2 A, A, B;\n\t"     // a = RN(acc * beta)
+        "mul.rn.f32x2 Q, A, Y;\n\t"     // q = RN(a * y)
+        "fma.rn.f32x2 R, Q, N, A;\n\t"  // a - q*s
+        "fma.rn.f32x2 Q, R, Y, Q;\n\t"  // q + (a - q*s)*y
+        "fma.rn.f32x2 R, Q, N, A;\n\t"  // exact remainder of the refined q
+        "mov.b64 {%0, %1}, Q;\n\t"
+        "mov.b64 {%2, %3}, R;\n\t}"
+        : "=f"(y0), "=f"(y1), "=f"(r0), "=f"(r1)
+        : "f"(__int2float_rn(a0)), "f"(__int2float_rn(a1)), "f"(beta), "f"(d.y), "f"(d.ns));
+    const uint32_t qb0 = __float_as_uint(y0), qb1 = __float_as_uint(y1);
+    const float h0 = __fmul_rn(__uint_as_float((qb0 & 0x7F800000u) - 0x0C000000u), d.s);
+    const float h1 = __fmul_rn(__uint_as_float((qb1 & 0x7F800000u) - 0x0C000000u), d.s);
+    ok0 = a0 == 0 || ((qb0 & 0x007FFFFFu) != 0u && fabsf(r0) < h0);
+    ok1 = a1 == 0 || ((qb1 & 0x007FFFFFu) != 0u && fabsf(r1) < h1);
+}
+
+// y[j] = RN32(RN32((v[j] - rsum) * beta) / s) for 16 outputs.
+__device__ __forceinline__ void scale16(const uint32_t* v, int rsum, float beta, const PairDiv& d,
+                                        float (&y)[16]) {
+    uint32_t bad = 0;
+#pragma unroll
+    for (int j = 0; j < 16; j += 2) {
+        bool ok0, ok1;
+        scale_fast2((int)v[j] - rsum, (int)v[j + 1] - rsum, beta, d, y[j], y[j + 1], ok0, ok1);
+        bad |= ((ok0 ? 0u : 1u) | (ok1 ? 0u : 2u)) << j;
+    }
+    if (!d.fast) bad = 0xFFFFu;
+    if (bad) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (bad & (1u << j)) y[j] = scale_slow((int)v[j] - rsum, beta, d.s, d.y);
+    }
+}
+
 // y = RN32(RN32(acc * beta) / s_x)
 __device__ __forceinline__ float tc_scale(int acc, float beta, const PairDiv& s_x) {
     return recip_div(__fmul_rn(__int2float_rn(acc), beta), RecipDiv{s_x.s, s_x.y});
