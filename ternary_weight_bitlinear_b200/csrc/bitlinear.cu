@@ -309,18 +309,30 @@ EncodeTiledFn encode_tiled() {
 
 // 2-D uint8 tensor [outer, inner] (row stride = inner bytes), tiles of
 // box_outer x box_inner; elements outside the tensor read as zero.
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType type, uint64_t elem_bytes, const void* ptr,
+                 uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swizzle);
+
 bool make_map_u8(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer,
                  uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+    return make_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, inner, outer, box_inner,
+                       box_outer, swizzle);
+}
+
+// 2-D tensor [outer, inner] of elem_bytes-wide elements, rows contiguous.
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType type, uint64_t elem_bytes, const void* ptr,
+                 uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swizzle) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) {
         snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled is unavailable");
         return false;
     }
     const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {inner};
+    const cuuint64_t strides[1] = {inner * elem_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims,
+    const CUresult r = fn(map, type, 2, const_cast<void*>(ptr), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -359,13 +371,22 @@ bl_status run_gemm(const int8_t* q, const float* s_x, const int32_t* rowsum, con
     a.vec_ok = ((N / 4) * out_bytes % 16 == 0) && (N * out_bytes % 16 == 0) &&
                (reinterpret_cast<uintptr_t>(y) % 16 == 0) &&
                (!residual || reinterpret_cast<uintptr_t>(residual) % 16 == 0);
+    // bf16 y without a residual leaves through TMA stores of 32 x 32 chunks
+    // (column offsets i*R + r are multiples of 8 elements when vec_ok holds)
+    CUtensorMap map_y = map_q;
+    if (a.vec_ok && epi == kEpiBF16 && !residual) {
+        if (!make_map_2d(&map_y, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, y, (uint64_t)N, (uint64_t)M, 32,
+                         32, CU_TENSOR_MAP_SWIZZLE_64B))
+            return BL_ERR_CUDA;
+        a.tma_store = 1;
+    }
     if (prepare_kernel(reinterpret_cast<const void*>(gemm_tc_kernel), dev, info, kTcThreads,
                        kTcSmemBytes) < 0)
         return BL_ERR_CUDA;
     const int64_t tiles = (int64_t)a.tiles_n * a.tiles_m;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(tiles, info.sms));
     return launch(gemm_tc_kernel, dim3((unsigned)grid), dim3(kTcThreads), (size_t)kTcSmemBytes,
-                  stream, map_q, map_p, a);
+                  stream, map_q, map_p, map_y, a);
 }
 
 // A launch epoch for the partial-sum flags: never 0 (a cleared flag), and

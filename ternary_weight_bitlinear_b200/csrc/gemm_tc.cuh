@@ -50,7 +50,10 @@ constexpr int kTcStageTx = kTcABytes + kTcPBytes;
 // layout from a 1024-aligned base: A[5] | B[2] | P[5] | barriers | tmem addr
 constexpr int kTcOffB = kTcStages * kTcABytes;
 constexpr int kTcOffP = kTcOffB + kTcExp * kTcBBytes;
-constexpr int kTcOffBar = kTcOffP + kTcStages * kTcPBytes;
+// per epilogue warp two 32 x 32 bf16 staging buffers for the TMA stores of y
+constexpr int kTcStageOut = 32 * 32 * 2;
+constexpr int kTcOffOut = kTcOffP + kTcStages * kTcPBytes;
+constexpr int kTcOffBar = kTcOffOut + 2 * 8 * kTcStageOut;
 constexpr int kTcNumBars = 2 * kTcStages + 2 * kTcExp + 5;
 constexpr int kTcOffTmem = kTcOffBar + 8 * kTcNumBars;
 constexpr int kTcSmemBytes = kTcOffTmem + 16 + 1024;   // + alignment slack
@@ -74,9 +77,27 @@ struct TcArgs {
     int tiles_n;               // ceil(R / 64)
     int tiles_m;               // ceil(M / 128)
     int vec_ok;                // outputs of 32 consecutive rows can use 16-byte accesses
+    int tma_store;             // bf16 y without residual: full 32 x 32 chunks leave by TMA store
 };
 
 // ---- tcgen05 / TMA wrappers ------------------------------------------------
+// Shared -> global tile store (TMA, bulk-group completion); rows or columns
+// outside the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(x), "r"(y)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most one of this thread's bulk stores still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read_1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+// Wait until this thread's bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar) {
     asm volatile(
@@ -277,7 +298,7 @@ __device__ __forceinline__ void tc_store_row32(const TcArgs& a, int64_t base, co
 
 __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
     const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_p,
-    const TcArgs a) {
+    const __grid_constant__ CUtensorMap tmap_y, const TcArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;  // 1024-aligned for the 128-byte swizzle
@@ -412,6 +433,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
         // ---------------- epilogue: one token per thread ----------------
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
         const int half = (warp - kTcEpiWarp0) >> 2;  // which 128 of the 256 columns
+        // this warp's two staging buffers (64-byte rows, 64-byte swizzle: chunk c
+        // of row r sits at chunk c ^ ((r >> 1) & 3))
+        uint8_t* stage = sm + kTcOffOut + (warp - kTcEpiWarp0) * 2 * kTcStageOut;
+        uint32_t nstore = 0;
         uint32_t tl = 0;
         for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tl) {
             const int tn = (int)(t / a.tiles_m), tm = (int)(t % a.tiles_m);
@@ -431,13 +456,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
                 const int i = c0 / kTcPackRows;                       // bit pair
                 const int r = tn * kTcPackRows + (c0 % kTcPackRows);  // first packed row
                 const int valid = min(32, a.R - r);
-                if (live && valid > 0)
+                if (a.tma_store && valid == 32) {
+                    // 32 tokens x 32 outputs: pack, stage, one TMA store (rows past M are dropped)
+                    uint32_t w[16];
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        float y[16];
+                        scale16(v + 16 * g, rsum, a.beta, sx, y);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) w[8 * g + j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
+                    }
+                    uint8_t* buf_out = stage + (nstore & 1) * kTcStageOut;
+                    if (lane == 0) bulk_wait_read_1();  // the store that used this buffer has read it
+                    __syncwarp();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4*>(buf_out + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+                            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0)
+                        tma_store_2d(&tmap_y, smem_addr(buf_out), i * a.R + r, tm * kTcBM + q * 32);
+                    ++nstore;
+                } else if (live && valid > 0) {
                     tc_store_row32(a, (int64_t)m * a.N + (int64_t)i * a.R + r, v, rsum, sx, valid);
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(accempty_bar(buf));
         }
+        if (lane == 0) bulk_wait_all();  // the stores are complete before the CTA's memory goes
     }
 
     tc_fence_before();
