@@ -385,6 +385,10 @@ bl_status run_gemm(const int8_t* q, const float* s_x, const int32_t* rowsum, con
         return BL_ERR_CUDA;
     const int64_t tiles = (int64_t)a.tiles_n * a.tiles_m;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(tiles, info.sms));
+    // a last wave less than half full runs as N-halves, twice as many units
+    const int64_t tail = tiles % grid;
+    a.full_units = (tiles > grid && tail > 0 && 2 * tail <= grid) ? tiles - tail : tiles;
+    a.units = a.full_units + 2 * (tiles - a.full_units);
     return launch(gemm_tc_kernel, dim3((unsigned)grid), dim3(kTcThreads), (size_t)kTcSmemBytes,
                   stream, map_q, map_p, map_y, a);
 }

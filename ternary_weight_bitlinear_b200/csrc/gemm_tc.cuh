@@ -8,7 +8,10 @@
 //
 // Tile: 128 tokens x 256 output rows (= 64 packed rows x 4 bit pairs), K in
 // stages of 128 bytes.  Persistent CTAs, one per SM, walk the tiles
-// round-robin.  Warp roles:
+// round-robin; when the last wave would fill at most half the SMs its tiles
+// run as two halves in N each (32 packed rows, MMA N=128), on twice as many
+// SMs.
+// Warp roles:
 //   warp 0      TMA producer: per stage, the 128x128-byte int8 activation tile
 //               (A operand, 128-byte swizzle, rows past M zero-filled) and the
 //               64x128-byte packed weight tile; no multicast.
@@ -26,6 +29,8 @@
 #pragma once
 
 #include <cuda.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "decode.cuh"
@@ -78,6 +83,27 @@ struct TcArgs {
     int tiles_m;               // ceil(M / 128)
     int vec_ok;                // outputs of 32 consecutive rows can use 16-byte accesses
     int tma_store;             // bf16 y without residual: full 32 x 32 chunks leave by TMA store
+    int64_t full_units;        // tiles processed whole; the rest as two N-halves each
+    int64_t units;             // full_units + 2 * (tiles - full_units)
+};
+
+// Work unit u of the round-robin schedule: a whole 128 x 256 tile, or (past
+// full_units) one half in N of a tile of the last partial wave -- 32 of its
+// 64 packed rows, 128 output rows -- so that wave's tiles spread over twice
+// as many SMs.
+struct TcUnit {
+    int tn, tm;
+    int nh;    // -1: whole tile; 0 / 1: packed rows 0-31 / 32-63 of it
+    __device__ __forceinline__ TcUnit(const TcArgs& a, int64_t u) {
+        int64_t t = u;
+        nh = -1;
+        if (u >= a.full_units) {
+            t = a.full_units + (u - a.full_units) / 2;
+            nh = (int)((u - a.full_units) & 1);
+        }
+        tn = (int)(t / a.tiles_m);
+        tm = (int)(t % a.tiles_m);
+    }
 };
 
 // ---- tcgen05 / TMA wrappers ------------------------------------------------
@@ -167,9 +193,11 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 }
 
 // Instruction descriptor: int32 accumulate, signed 8-bit A and B, both
-// K-major, M = kTcBM, N = kTcBN.
+// K-major, M = kTcBM, N = kTcBN (or half of it for a half unit).
 constexpr uint32_t kTcIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTcBN >> 3) << 17) |
                               ((uint32_t)(kTcBM >> 4) << 24);
+constexpr uint32_t kTcIdescHalf = (2u << 4) | (1u << 7) | (1u << 10) |
+                                  ((uint32_t)(kTcBN / 2 >> 3) << 17) | ((uint32_t)(kTcBM >> 4) << 24);
 
 // Byte offset of the 16-byte chunk `chunk16` of `row` in a 128-byte-wide,
 // 128-byte-swizzled K-major tile (8-row groups of 1024 bytes).
@@ -296,6 +324,26 @@ __device__ __forceinline__ void tc_store_row32(const TcArgs& a, int64_t base, co
     }
 }
 
+// Expand one stage of packed codes into the B operand: packed row rr, bit
+// pair i -> B row i * rows + rr (rows = 64 packed rows, or the 32 of a half
+// unit starting at pk), codes t + 1 as int8 in the 128-byte swizzle.
+template <bool kHalf>
+__device__ __forceinline__ void tc_expand(const uint8_t* pk, uint8_t* bt, int e0) {
+    constexpr int rows = kHalf ? kTcPackRows / 2 : kTcPackRows;
+#pragma unroll
+    for (int it = 0; it < rows * 8 / (32 * kTcExpWarps); ++it) {
+        const int item = e0 + it * 32 * kTcExpWarps;  // (packed row, 16-byte chunk)
+        const int rr = item >> 3, ch = item & 7;
+        const uint4 w = *reinterpret_cast<const uint4*>(pk + rr * kTcBK + ch * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 c = make_uint4((w.x >> (2 * i)) & 0x03030303u, (w.y >> (2 * i)) & 0x03030303u,
+                                       (w.z >> (2 * i)) & 0x03030303u, (w.w >> (2 * i)) & 0x03030303u);
+            *reinterpret_cast<uint4*>(bt + sw128_offset(i * rows + rr, ch)) = c;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
     const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_p,
     const __grid_constant__ CUtensorMap tmap_y, const TcArgs a) {
@@ -340,7 +388,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
     pdl_wait();
     pdl_launch_dependents();
 
-    const int64_t tiles = (int64_t)a.tiles_n * a.tiles_m;
     const int kstages = (a.K + kTcBK - 1) / kTcBK;
     bool ok = true;
 
@@ -349,8 +396,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
         if (lane == 0) {
             uint32_t g = 0;
             uint32_t inflight_from = 0;  // stages [inflight_from, g) may still be landing
-            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                const int tn = (int)(t / a.tiles_m), tm = (int)(t % a.tiles_m);
+            for (int64_t u = blockIdx.x; u < a.units && ok; u += gridDim.x) {
+                const TcUnit un(a, u);
+                const int tn = un.tn, tm = un.tm;
                 for (int ks = 0; ks < kstages; ++ks, ++g) {
                     const int s = (int)(g % kTcStages);
                     if (!mbar_wait(empty_bar(s), ((g / kTcStages) & 1u) ^ 1u)) { ok = false; break; }
@@ -369,39 +417,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
         // ---------------- expansion: 2-bit codes -> int8 B tile ----------------
         const int e0 = threadIdx.x - 32;  // 0 .. 32*kTcExpWarps-1
         uint32_t g = 0;
-        for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        // one instantiation of the stage loop per unit kind keeps the whole-tile loop branch-free
+        auto expand_unit = [&](auto half_tag, const int rr0) {
+            constexpr bool kHalf = decltype(half_tag)::value;
             for (int ks = 0; ks < kstages; ++ks, ++g) {
                 const int s = (int)(g % kTcStages), e = (int)(g % kTcExp);
                 const bool got = mbar_wait(full_bar(s), (g / kTcStages) & 1u) &&
                                  mbar_wait(bfree_bar(e), ((g / kTcExp) & 1u) ^ 1u);
-                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-                const uint8_t* pk = sm + kTcOffP + s * kTcPBytes;
-                uint8_t* bt = sm + kTcOffB + e * kTcBBytes;
-#pragma unroll
-                for (int it = 0; it < kTcPackRows * 8 / (32 * kTcExpWarps); ++it) {
-                    const int item = e0 + it * 32 * kTcExpWarps;  // (packed row, 16-byte chunk)
-                    const int rr = item >> 3, ch = item & 7;
-                    const uint4 w = *reinterpret_cast<const uint4*>(pk + rr * kTcBK + ch * 16);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int row = i * kTcPackRows + rr;
-                        const uint4 c = make_uint4((w.x >> (2 * i)) & 0x03030303u,
-                                                   (w.y >> (2 * i)) & 0x03030303u,
-                                                   (w.z >> (2 * i)) & 0x03030303u,
-                                                   (w.w >> (2 * i)) & 0x03030303u);
-                        *reinterpret_cast<uint4*>(bt + sw128_offset(row, ch)) = c;
-                    }
-                }
+                if (!__all_sync(0xffffffffu, got)) return false;
+                tc_expand<kHalf>(sm + kTcOffP + s * kTcPBytes + rr0 * kTcBK, sm + kTcOffB + e * kTcBBytes, e0);
                 fence_proxy_async_smem();  // generic writes -> visible to the tensor core
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bready_bar(e));
             }
+            return true;
+        };
+        for (int64_t u = blockIdx.x; u < a.units && ok; u += gridDim.x) {
+            const TcUnit un(a, u);
+            ok = un.nh < 0 ? expand_unit(std::false_type{}, 0)
+                           : expand_unit(std::true_type{}, un.nh * (kTcPackRows / 2));
         }
     } else if (warp == kTcMmaWarp) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             uint32_t g = 0, tl = 0;
-            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tl) {
+            for (int64_t u = blockIdx.x; u < a.units && ok; u += gridDim.x, ++tl) {
+                const uint32_t idesc = u >= a.full_units ? kTcIdescHalf : kTcIdesc;
                 const int buf = (int)(tl & 1);
                 if (!mbar_wait(accempty_bar(buf), ((tl >> 1) & 1u) ^ 1u)) { ok = false; break; }
                 tc_fence_after();
@@ -418,7 +459,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
                     const uint64_t bd = smem_desc_sw128(sB + e * kTcBBytes);
 #pragma unroll
                     for (int kk = 0; kk < kTcBK / 32; ++kk)  // +32 bytes = +2 in the address field
-                        tc_mma_i8(d, ad + 2u * kk, bd + 2u * kk, kTcIdesc, (ks | kk) != 0);
+                        tc_mma_i8(d, ad + 2u * kk, bd + 2u * kk, idesc, (ks | kk) != 0);
                     tc_commit(empty_bar(s));  // activation + packed stage reusable
                     tc_commit(bfree_bar(e));  // expanded operand reusable
                 }
@@ -438,8 +479,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
         uint8_t* stage = sm + kTcOffOut + (warp - kTcEpiWarp0) * 2 * kTcStageOut;
         uint32_t nstore = 0;
         uint32_t tl = 0;
-        for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tl) {
-            const int tn = (int)(t / a.tiles_m), tm = (int)(t % a.tiles_m);
+        for (int64_t u = blockIdx.x; u < a.units && ok; u += gridDim.x, ++tl) {
+            const TcUnit un(a, u);
+            const int tn = un.tn, tm = un.tm;
+            // columns of this warp: [cb, ce) of the unit's 256 (whole) or 128 (half);
+            // column c is bit pair c >> lg of packed row tn * 64 + rr0 + (c & (2^lg - 1))
+            const int ucols = un.nh < 0 ? kTcBN : kTcBN / 2;
+            const int cb = half * (ucols / 2), ce = cb + ucols / 2;
+            const int lg = un.nh < 0 ? 6 : 5;
+            const int rr0 = un.nh < 0 ? 0 : un.nh * (kTcPackRows / 2);
             const int buf = (int)(tl & 1);
             const int m = tm * kTcBM + q * 32 + lane;  // this thread's token
             const bool live = m < a.M;
@@ -450,11 +498,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kTcBN);
 #pragma unroll 1
-            for (int c0 = half * (kTcBN / 2); c0 < (half + 1) * (kTcBN / 2); c0 += 32) {
+            for (int c0 = cb; c0 < ce; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld32(taddr + (uint32_t)c0, v);
-                const int i = c0 / kTcPackRows;                       // bit pair
-                const int r = tn * kTcPackRows + (c0 % kTcPackRows);  // first packed row
+                const int i = c0 >> lg;                                          // bit pair
+                const int r = tn * kTcPackRows + rr0 + (c0 & ((1 << lg) - 1));  // first packed row
                 const int valid = min(32, a.R - r);
                 if (a.tma_store && valid == 32) {
                     // 32 tokens x 32 outputs: pack, stage, one TMA store (rows past M are dropped)

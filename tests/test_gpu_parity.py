@@ -362,6 +362,10 @@ def test_batch_of_many_tiny_problems_and_one_large():
     (257, 128, 256, "bf16", False),    # exactly one K stage, one weight tile
     (1000, 2560, 6912, "bf16", True),  # 216 tiles > 148 CTAs: both accumulators reused
     (130, 6912, 2560, "i32", False),   # exact int32 accumulators, 54 K stages
+    # last wave split in N: 160 tiles on 148 CTAs leave 12 tiles for 24 halves
+    (256, 128, 20304, "bf16", False),  # R=5076: last tile 20 rows, its second half empty
+    (256, 144, 20384, "f32", False),   # R=5096: second half of the last tile 8 rows
+    (200, 256, 20480, "i32", False),   # R=5120: every half full, int32 accumulators
 ])
 def test_gemm_path_shapes(M, K, N, out, residual):
     x = special_rows(WL.activations(M, K, seed=M * 7 + K, row_std=(0.1, 10.0)))
