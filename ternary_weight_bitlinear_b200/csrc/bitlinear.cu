@@ -29,8 +29,9 @@ using namespace bl;
 constexpr int kQuantThreads = 256;
 constexpr int kSmallBatch = 8;  // parameter-table size of small batches
 constexpr int64_t kQuantWarpMinRows = 1024;  // rows from which a warp per row pays off
-constexpr int kQuantRegVpt1 = 10;  // 16-byte vectors per thread, one warp per row: K <= 2560
-constexpr int kQuantRegVpt4 = 7;   // ... four warps per row: K <= 7168
+// many rows: one CTA of W warps per row, VPT 16-byte vectors per thread
+constexpr int kQuantRowW1 = 2, kQuantRowVpt1 = 5;  // K <= 2560
+constexpr int kQuantRowW2 = 8, kQuantRowVpt2 = 4;  // K <= 8192
 
 // ---- device properties and per-kernel launch settings ---------------------
 struct DeviceInfo {
@@ -178,19 +179,19 @@ bl_status launch_quant_cap(const QuantProblem* probs, int count, int64_t M, floa
         kmax = std::max(kmax, probs[i].K);
     }
     const int64_t rows = (int64_t)count * M;
-    if (rows >= kQuantWarpMinRows && kmax <= 32 * 8 * kQuantRegVpt1) {
-        // many rows (prefill), short rows: one warp per row, held in registers
-        auto fn = quant_reg_kernel<1, kQuantRegVpt1, CAP>;
-        if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, 128, 0) < 0)
+    if (rows >= kQuantWarpMinRows && kmax <= 8 * 32 * kQuantRowW1 * kQuantRowVpt1) {
+        // many rows (prefill), rows up to 2560: two warps per row, held in registers
+        auto fn = quant_row_kernel<kQuantRowW1, kQuantRowVpt1, CAP>;
+        if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, 32 * kQuantRowW1, 0) < 0)
             return BL_ERR_CUDA;
-        return launch(fn, dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, stream, b);
+        return launch(fn, dim3((unsigned)rows), dim3(32 * kQuantRowW1), 0, stream, b);
     }
-    if (rows >= kQuantWarpMinRows && kmax <= 128 * 8 * kQuantRegVpt4) {
-        // many rows, longer rows: four warps per row, held in registers
-        auto fn = quant_reg_kernel<4, kQuantRegVpt4, CAP>;
-        if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, 128, 0) < 0)
+    if (rows >= kQuantWarpMinRows && kmax <= 8 * 32 * kQuantRowW2 * kQuantRowVpt2) {
+        // many rows, longer rows: eight warps per row, held in registers
+        auto fn = quant_row_kernel<kQuantRowW2, kQuantRowVpt2, CAP>;
+        if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, 32 * kQuantRowW2, 0) < 0)
             return BL_ERR_CUDA;
-        return launch(fn, dim3((unsigned)rows), dim3(128), 0, stream, b);
+        return launch(fn, dim3((unsigned)rows), dim3(32 * kQuantRowW2), 0, stream, b);
     }
     if (kmax <= kQuantWarpMaxK && rows >= kQuantWarpMinRows) {
         // many rows (prefill): one warp per row, up to 8 rows per CTA; few rows

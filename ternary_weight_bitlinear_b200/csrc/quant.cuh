@@ -381,59 +381,80 @@ __global__ void __launch_bounds__(256) quant_warp_kernel(const __grid_constant__
     }
 }
 
-// ---- rows held in registers: W warps per row, up to VPT vectors per thread ----
+// ---- many rows: one row per CTA of W warps, the row held in registers ----
 // Same arithmetic as quantize_row.  Every 16-byte load of the row is issued
-// before any use, so a thread has VPT loads in flight; nothing is staged in
-// shared memory.  W = 1: one warp per row (4 rows per CTA, no block barriers);
-// W = 4: one CTA per row (K up to 128 * 8 * VPT).
+// before any use (VPT per thread); the values are unpacked once to fp32
+// (exact for bf16) and the RMSNorm pass overwrites them with the normalised
+// h, which the code pass reads; nothing is staged in shared memory.
+//
+// Codes: |h * s_x| <= 127 (1 + 2^-24) for every element of the row (s_x is
+// RN32(127 / max(max|h|, 1e-5))), so RN32(h * s_x) rounds to an integer c in
+// [-127, 127] and the clamp to [-128, 127] never binds.  c is taken by the
+// add-magic-number method: for |v| < 2^22, RN32(v + 1.5 * 2^23) lies in
+// [2^23, 2^24), where the ulp is 1, so the IEEE addition itself rounds v to
+// the nearest integer, ties to even, and the sum's bits are 0x4B400000 + c
+// (low byte: c as an int8).  Activations are assumed finite.
+constexpr uint32_t kMagicBits = 0x4B400000u;  // bits of 1.5 * 2^23
+
 template <int W, int VPT, int CAP>
-__global__ void __launch_bounds__(128, 4) quant_reg_kernel(const __grid_constant__ QuantBatch<CAP> b) {
-    static_assert(W == 1 || W == 4, "one warp or one CTA per row");
-    constexpr int RPC = 4 / W;  // rows per CTA
-    constexpr int NTR = 32 * W; // threads per row
-    __shared__ double red_hi[4], red_lo[4];
-    __shared__ float red_f[4];
-    __shared__ int red_i[4];
+__global__ void __launch_bounds__(32 * W, 24 / W) quant_row_kernel(const __grid_constant__ QuantBatch<CAP> b) {
+    static_assert(W >= 1 && W <= 8 && 24 % W == 0, "1 to 8 warps per row");
+    constexpr int NTR = 32 * W;  // threads per row
+    __shared__ double red_d[2][W];
+    __shared__ float red_f[W];
+    __shared__ int red_i[W];
     pdl_launch_dependents();
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int sub = warp % W;
-    const int row = blockIdx.x * RPC + warp / W;
-    if (row >= b.count * b.M) return;  // uniform over a row's warps; W = 4: over the CTA
+    const int row = blockIdx.x;
     const int p = row / b.M, m = row % b.M;
     const QuantProblem pr = b.p[p];
-    const int t = sub * 32 + lane;
+    const int t = threadIdx.x;
     const int nvec = pr.K >> 3;
     const uint4* xv = reinterpret_cast<const uint4*>(pr.x + (int64_t)m * pr.K);
     const uint4* gv = reinterpret_cast<const uint4*>(pr.gain);
     const bool norm = pr.gain != nullptr;
 
-    uint4 xr[VPT];
+    float h[VPT][8];
+    {
+        uint4 xr[VPT];
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        const int v = t + i * NTR;
-        xr[i] = v < nvec ? __ldcg(xv + v) : make_uint4(0u, 0u, 0u, 0u);  // zeros add nothing
+        for (int i = 0; i < VPT; ++i) {
+            const int v = t + i * NTR;
+            xr[i] = v < nvec ? __ldcg(xv + v) : make_uint4(0u, 0u, 0u, 0u);  // zeros add nothing
+        }
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) unpack8_bf16(xr[i], h[i]);
     }
 
-    // sum over the row's threads, in a fixed order (W = 4: warps in index order)
-    auto row_sum_dd = [&](double hi, double lo) -> double {
+    // reductions over the row's threads: shuffle tree, then warps in index order
+    auto row_sum_d = [&](double v) -> double {  // plain binary64 additions
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (W == 1) return v;
+        if (lane == 0) red_d[0][warp] = v;
+        __syncthreads();
+        double r = red_d[0][0];
+        for (int w = 1; w < W; ++w) r = __dadd_rn(r, red_d[0][w]);
+        __syncthreads();
+        return r;
+    };
+    auto row_sum_dd = [&](double hi, double lo) -> double {  // (hi, lo) pairs, error-free merges
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const double ohi = __shfl_down_sync(0xffffffffu, hi, o);
             const double olo = __shfl_down_sync(0xffffffffu, lo, o);
             if (lane < o) dd_merge(hi, lo, ohi, olo);
         }
-        if (W == 1) {
-            hi = __shfl_sync(0xffffffffu, hi, 0);
-            lo = __shfl_sync(0xffffffffu, lo, 0);
-            return __dadd_rn(hi, lo);
-        }
-        if (lane == 0) { red_hi[warp] = hi; red_lo[warp] = lo; }
+        hi = __shfl_sync(0xffffffffu, hi, 0);
+        lo = __shfl_sync(0xffffffffu, lo, 0);
+        if (W == 1) return __dadd_rn(hi, lo);
+        if (lane == 0) { red_d[0][warp] = hi; red_d[1][warp] = lo; }
         __syncthreads();
-        double h = red_hi[0], l = red_lo[0];
-        for (int w = 1; w < W; ++w) dd_merge(h, l, red_hi[w], red_lo[w]);
+        double rh = red_d[0][0], rl = red_d[1][0];
+        for (int w = 1; w < W; ++w) dd_merge(rh, rl, red_d[0][w], red_d[1][w]);
         __syncthreads();
-        return __dadd_rn(h, l);
+        return __dadd_rn(rh, rl);
     };
     auto row_max = [&](float v) -> float {
 #pragma unroll
@@ -443,7 +464,7 @@ __global__ void __launch_bounds__(128, 4) quant_reg_kernel(const __grid_constant
         __syncthreads();
         float r = red_f[0];
         for (int w = 1; w < W; ++w) r = fmaxf(r, red_f[w]);
-        return r;  // the next barrier (in row_sum_int) orders the reuse of red_f
+        return r;
     };
     auto row_sum_int = [&](int v) -> int {
 #pragma unroll
@@ -456,21 +477,18 @@ __global__ void __launch_bounds__(128, 4) quant_reg_kernel(const __grid_constant
         return r;
     };
 
-    float r = 1.0f, mx = 0.0f;
+    float mx = 0.0f;
     if (norm) {
-        double ss0 = 0.0, ss1 = 0.0;  // plain binary64 sums of the exact squares
+        double ss0 = 0.0, ss1 = 0.0;  // binary64 sums of the exact squares
 #pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            float f[8];
-            unpack8_bf16(xr[i], f);
+        for (int i = 0; i < VPT; ++i)
 #pragma unroll
             for (int j = 0; j < 8; j += 2) {
-                ss0 = __fma_rn((double)f[j], (double)f[j], ss0);
-                ss1 = __fma_rn((double)f[j + 1], (double)f[j + 1], ss1);
+                ss0 = __fma_rn((double)h[i][j], (double)h[i][j], ss0);
+                ss1 = __fma_rn((double)h[i][j + 1], (double)h[i][j + 1], ss1);
             }
-        }
-        const double approx = row_sum_dd(__dadd_rn(ss0, ss1), 0.0);
-        if (!rms_factor_bounded(approx, pr.K, b.eps, r)) {
+        float r;
+        if (!rms_factor_bounded(row_sum_d(__dadd_rn(ss0, ss1)), pr.K, b.eps, r)) {
             // rare: the interval straddles a rounding boundary; take the sum
             // exactly (re-reading the row from L2 keeps this path's registers
             // away from the common one)
@@ -491,53 +509,44 @@ __global__ void __launch_bounds__(128, 4) quant_reg_kernel(const __grid_constant
         for (int i = 0; i < VPT; ++i) {
             const int v = t + i * NTR;
             if (v < nvec) {
-                float f[8], g[8];
-                unpack8_bf16(xr[i], f);
+                float g[8];
                 unpack8_bf16(__ldg(gv + v), g);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(norm_elem(f[j], r, g[j])));
+                for (int j = 0; j < 8; ++j) {
+                    h[i][j] = norm_elem(h[i][j], r, g[j]);
+                    mx = fmaxf(mx, fabsf(h[i][j]));
+                }
             }
         }
     } else {
 #pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            float f[8];
-            unpack8_bf16(xr[i], f);
+        for (int i = 0; i < VPT; ++i)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(f[j]));
-        }
+            for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(h[i][j]));
     }
     const float s = __fdiv_rn(127.0f, fmaxf(row_max(mx), kScaleFloor));
 
-    int rs = 0;
+    uint32_t rs = 0;  // sum of (magic bits - kMagicBits), modulo 2^32: the row sum fits
     int8_t* q = pr.q + (int64_t)m * pr.K;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
         const int v = t + i * NTR;
         if (v < nvec) {
-            float f[8];
-            unpack8_bf16(xr[i], f);
-            if (norm) {
-                float g[8];
-                unpack8_bf16(__ldg(gv + v), g);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] = norm_elem(f[j], r, g[j]);
-            }
-            uint32_t packed[2] = {0u, 0u};
+            uint32_t c[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                int c = __float2int_rn(__fmul_rn(f[j], s));  // round half to even
-                c = min(max(c, -128), 127);
-                rs += c;
-                packed[j >> 2] |= (uint32_t)(c & 0xFF) << (8 * (j & 3));
+                c[j] = __float_as_uint(__fadd_rn(__fmul_rn(h[i][j], s), 12582912.0f));
+                rs += c[j] - kMagicBits;
             }
-            reinterpret_cast<uint2*>(q)[v] = make_uint2(packed[0], packed[1]);
+            const uint32_t lo = __byte_perm(__byte_perm(c[0], c[1], 0x0040u), __byte_perm(c[2], c[3], 0x0040u), 0x5410u);
+            const uint32_t hi = __byte_perm(__byte_perm(c[4], c[5], 0x0040u), __byte_perm(c[6], c[7], 0x0040u), 0x5410u);
+            reinterpret_cast<uint2*>(q)[v] = make_uint2(lo, hi);
         }
     }
-    rs = row_sum_int(rs);
+    const int rsum = row_sum_int((int)rs);
     if (t == 0) {
         pr.s_x[m] = s;
-        if (pr.rowsum) pr.rowsum[m] = rs;
+        if (pr.rowsum) pr.rowsum[m] = rsum;
     }
 }
 

@@ -100,17 +100,39 @@ def special_rows(x):
 
 @pytest.mark.parametrize("norm", [False, True])
 @pytest.mark.parametrize("M,K", [(1, 16), (3, 256), (4, 2560), (7, 6912), (64, 2560), (257, 272),
-                                 # 1024+ rows: the register-resident kernels (one warp per
-                                 # row up to K = 2560, four up to 7168) and, past that, the
+                                 # 1024+ rows: the register-resident kernels (two warps per
+                                 # row up to K = 2560, eight up to 8192) and, past that, the
                                  # shared-memory warp kernel
                                  (1024, 2560), (1031, 6912), (1100, 272), (1024, 2576),
-                                 (1025, 7168), (1024, 8192)])
+                                 (1025, 7168), (1024, 8192), (1030, 8208)])
 def test_act_quant_matches_oracle(M, K, norm):
     x = special_rows(WL.activations(M, K, seed=M * 131 + K, outlier_frac=0.001))
     gain = WL.gain(K, seed=K) if norm else None
     q, s, rs = B.bitlinear_act_quant(bf16_dev(x), None if gain is None else bf16_dev(gain),
                                      WL.RMS_EPS)
     q_o, s_o, rs_o = O.quantize_input(x, gain, WL.RMS_EPS, norm=norm)
+    assert_exact(s.cpu().numpy().view(np.uint32), s_o.view(np.uint32), "s_x")
+    assert_exact(q.cpu().numpy(), q_o, "codes")
+    assert_exact(rs.cpu().numpy(), rs_o, "row sums")
+
+
+@pytest.mark.parametrize("M,K", [(8, 2560),      # one CTA per row
+                                 (1024, 2560),   # many rows: two warps per row
+                                 (1031, 6912),   # eight warps per row
+                                 (1024, 8208),   # past 8192: the shared-memory warp kernel
+                                 (1, 16)])
+def test_act_quant_rms_boundary_rows(M, K):
+    """Rows whose RMSNorm factor is decided by the rounding of the exact sum of
+    squares (the fast interval test must fall back to the exact sum) at
+    several places of the batch."""
+    from rms_boundary import straddle_rows
+    x = WL.activations(M, K, seed=M * 7 + K)
+    n = min(M, 8)
+    at = np.linspace(0, M - 1, n).astype(int)
+    x[at] = straddle_rows(n, K, WL.RMS_EPS, seed=K + M)
+    gain = WL.gain(K, seed=K + 1)
+    q, s, rs = B.bitlinear_act_quant(bf16_dev(x), bf16_dev(gain), WL.RMS_EPS)
+    q_o, s_o, rs_o = O.quantize_input(x, gain, WL.RMS_EPS, norm=True)
     assert_exact(s.cpu().numpy().view(np.uint32), s_o.view(np.uint32), "s_x")
     assert_exact(q.cpu().numpy(), q_o, "codes")
     assert_exact(rs.cpu().numpy(), rs_o, "row sums")

@@ -294,6 +294,21 @@ def test_rmsnorm_factor_exact(O):
         np.testing.assert_array_equal(h[m], (xf[m] * r[m]).astype(np.float32))
 
 
+@pytest.mark.parametrize("K", [16, 256, 2560])
+def test_rmsnorm_factor_on_rounding_boundaries(O, K):
+    """Rows whose exact sum of squares sits where RN64 of it decides between two
+    binary32 factors: the oracle gives the factor of the exact sum, and a plain
+    binary64 running sum of the same squares misses at least one of them."""
+    from rms_boundary import exact_sum_squares, factor_from_sum, straddle_rows
+    rows = straddle_rows(8, K, 1e-5, seed=K + 7)
+    _, r = O.rmsnorm(rows, None, 1e-5)
+    exact = np.array([factor_from_sum(float(exact_sum_squares(b)), K, 1e-5) for b in rows])
+    np.testing.assert_array_equal(r, exact)
+    xf = O.bf16_to_f32(rows).astype(np.float64)
+    running = np.array([factor_from_sum(float(np.cumsum(v * v)[-1]), K, 1e-5) for v in xf])
+    assert (running != exact).any()
+
+
 def test_rmsnorm_matches_textbook_formula(O):
     rng = np.random.default_rng(22)
     K = 2560
