@@ -29,9 +29,10 @@ using namespace bl;
 constexpr int kQuantThreads = 256;
 constexpr int kSmallBatch = 8;  // parameter-table size of small batches
 constexpr int64_t kQuantWarpMinRows = 1024;  // rows from which a warp per row pays off
-// many rows: one CTA of W warps per row, VPT 16-byte vectors per thread
-constexpr int kQuantRowW1 = 2, kQuantRowVpt1 = 5;  // K <= 2560
-constexpr int kQuantRowW2 = 8, kQuantRowVpt2 = 4;  // K <= 8192
+// many rows: one CTA of W warps per row, VPT 16-byte vectors per thread, at
+// least MINB CTAs per SM (the register budget)
+constexpr int kQuantRowW1 = 2, kQuantRowVpt1 = 5, kQuantRowMinB1 = 12;  // K <= 2560
+constexpr int kQuantRowW2 = 4, kQuantRowVpt2 = 7, kQuantRowMinB2 = 4;   // K <= 7168
 
 // ---- device properties and per-kernel launch settings ---------------------
 struct DeviceInfo {
@@ -181,14 +182,14 @@ bl_status launch_quant_cap(const QuantProblem* probs, int count, int64_t M, floa
     const int64_t rows = (int64_t)count * M;
     if (rows >= kQuantWarpMinRows && kmax <= 8 * 32 * kQuantRowW1 * kQuantRowVpt1) {
         // many rows (prefill), rows up to 2560: two warps per row, held in registers
-        auto fn = quant_row_kernel<kQuantRowW1, kQuantRowVpt1, CAP>;
+        auto fn = quant_row_kernel<kQuantRowW1, kQuantRowVpt1, kQuantRowMinB1, CAP>;
         if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, 32 * kQuantRowW1, 0) < 0)
             return BL_ERR_CUDA;
         return launch(fn, dim3((unsigned)rows), dim3(32 * kQuantRowW1), 0, stream, b);
     }
     if (rows >= kQuantWarpMinRows && kmax <= 8 * 32 * kQuantRowW2 * kQuantRowVpt2) {
-        // many rows, longer rows: eight warps per row, held in registers
-        auto fn = quant_row_kernel<kQuantRowW2, kQuantRowVpt2, CAP>;
+        // many rows, longer rows: four warps per row, held in registers
+        auto fn = quant_row_kernel<kQuantRowW2, kQuantRowVpt2, kQuantRowMinB2, CAP>;
         if (prepare_kernel(reinterpret_cast<const void*>(fn), dev, info, 32 * kQuantRowW2, 0) < 0)
             return BL_ERR_CUDA;
         return launch(fn, dim3((unsigned)rows), dim3(32 * kQuantRowW2), 0, stream, b);

@@ -396,9 +396,9 @@ __global__ void __launch_bounds__(256) quant_warp_kernel(const __grid_constant__
 // (low byte: c as an int8).  Activations are assumed finite.
 constexpr uint32_t kMagicBits = 0x4B400000u;  // bits of 1.5 * 2^23
 
-template <int W, int VPT, int CAP>
-__global__ void __launch_bounds__(32 * W, 24 / W) quant_row_kernel(const __grid_constant__ QuantBatch<CAP> b) {
-    static_assert(W >= 1 && W <= 8 && 24 % W == 0, "1 to 8 warps per row");
+template <int W, int VPT, int MINB, int CAP>
+__global__ void __launch_bounds__(32 * W, MINB) quant_row_kernel(const __grid_constant__ QuantBatch<CAP> b) {
+    static_assert(W >= 1 && W <= 8, "1 to 8 warps per row");
     constexpr int NTR = 32 * W;  // threads per row
     __shared__ double red_d[2][W];
     __shared__ float red_f[W];

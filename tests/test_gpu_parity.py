@@ -101,7 +101,7 @@ def special_rows(x):
 @pytest.mark.parametrize("norm", [False, True])
 @pytest.mark.parametrize("M,K", [(1, 16), (3, 256), (4, 2560), (7, 6912), (64, 2560), (257, 272),
                                  # 1024+ rows: the register-resident kernels (two warps per
-                                 # row up to K = 2560, eight up to 8192) and, past that, the
+                                 # row up to K = 2560, four up to 7168) and, past that, the
                                  # shared-memory warp kernel
                                  (1024, 2560), (1031, 6912), (1100, 272), (1024, 2576),
                                  (1025, 7168), (1024, 8192), (1030, 8208)])
@@ -118,8 +118,8 @@ def test_act_quant_matches_oracle(M, K, norm):
 
 @pytest.mark.parametrize("M,K", [(8, 2560),      # one CTA per row
                                  (1024, 2560),   # many rows: two warps per row
-                                 (1031, 6912),   # eight warps per row
-                                 (1024, 8208),   # past 8192: the shared-memory warp kernel
+                                 (1031, 6912),   # four warps per row
+                                 (1024, 8208),   # past 7168: the shared-memory warp kernel
                                  (1, 16)])
 def test_act_quant_rms_boundary_rows(M, K):
     """Rows whose RMSNorm factor is decided by the rounding of the exact sum of
