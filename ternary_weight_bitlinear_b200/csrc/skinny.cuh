@@ -35,8 +35,9 @@
 //    A row tile whose items straddle two or more CTAs is finished by the CTA
 //    holding its first items (it reaches them last): the others leave int32
 //    partial sums in the caller's workspace and raise a flag carrying this
-//    launch's epoch; the finisher adds them and clears the flags.  Without a
-//    workspace the CTA shares are cut at row-tile boundaries instead.
+//    launch's epoch; the finisher polls those flags side by side, adds the
+//    sums (16-byte loads of each contributor's block) and clears the flags.
+//    Without a workspace the CTA shares are cut at row-tile boundaries.
 //  * Every wait is bounded (status word + unwind).
 #pragma once
 
@@ -108,7 +109,7 @@ struct alignas(64) SkBatch {
     int64_t total;               // items in the batch
     unsigned long long epoch;    // nonzero, distinct per launch
     unsigned long long* flags;   // [gridDim.x] partial-sum flags (split only)
-    int32_t* part;               // [gridDim.x][npad][128] partial sums (split only)
+    int32_t* part;               // [gridDim.x][128][npad] partial sums (split only)
 };
 
 __device__ __forceinline__ int sk_problem_at(const SkBatch& b, int64_t item) {
@@ -446,14 +447,15 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(32 * qd) << 16) + kSkDCol0 + (uint32_t)d * kSkDBuf;
             // a finisher first waits for the partial sums of every later CTA
-            // whose share starts inside this tile (CTAs c+1 .. c_end-1)
+            // whose share starts inside this tile (CTAs c+1 .. c_end-1); the
+            // lanes of the first epilogue warp poll those flags side by side
             int64_t c_end = c + 1;
             bool waited = true;
             if (!started_before && continues) {
                 while (c_end < G && sk_share_start(b, c_end, G) < tile_end) ++c_end;
-                for (int64_t c2 = c + 1; c2 < c_end && waited; ++c2) {
-                    if (threadIdx.x == kSkEpiWarp0 * 32) {
-                        const unsigned long long t0 = globaltimer_ns();
+                if (warp == kSkEpiWarp0) {
+                    const unsigned long long t0 = globaltimer_ns();
+                    for (int64_t c2 = c + 1 + lane; c2 < c_end && waited; c2 += 32) {
                         while (ld_acquire_u64(b.flags + c2) != b.epoch) {
                             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                                 atomicOr(&g_status, kStatusTimeout);
@@ -462,8 +464,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
                             }
                         }
                     }
-                    waited = sk_epi_all(waited);  // also orders the flag before the reads
                 }
+                waited = sk_epi_all(waited);  // also orders the flags before the reads
             }
             const int r = cur.tile * kSkRows + 8 * qd + j;  // packed row
             const int64_t n = (int64_t)bit * pr.R + r;
@@ -478,17 +480,29 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
                     for (int m = 0; m < 32; ++m) v[m] += u[m];
                 }
                 if (started_before) {
-                    // contributor: leave the partial sums for the tile's finisher
-                    int32_t* dst = b.part + (size_t)c * b.npad * 128;
+                    // contributor: leave the partial sums for the tile's finisher,
+                    // each weight row's npad sums contiguous (16-byte stores)
+                    uint4* dst = reinterpret_cast<uint4*>(b.part + ((size_t)c * 128 + row128) * b.npad + 32 * h);
 #pragma unroll
-                    for (int m = 0; m < 32; ++m)
-                        if (32 * h + m < b.npad) dst[(32 * h + m) * 128 + row128] = (int32_t)v[m];
+                    for (int k = 0; k < 8; ++k)
+                        if (32 * h + 4 * k < b.npad)
+                            dst[k] = make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
                 } else if (waited) {
+                    // one contributor at a time, all of its 16-byte loads in flight
                     for (int64_t c2 = c + 1; c2 < c_end; ++c2) {
-                        const int32_t* src = b.part + (size_t)c2 * b.npad * 128;
+                        const uint4* src =
+                            reinterpret_cast<const uint4*>(b.part + ((size_t)c2 * 128 + row128) * b.npad + 32 * h);
+                        uint4 w[8];
 #pragma unroll
-                        for (int m = 0; m < 32; ++m)
-                            if (32 * h + m < b.npad) v[m] += (uint32_t)__ldcg(src + (32 * h + m) * 128 + row128);
+                        for (int k = 0; k < 8; ++k)
+                            w[k] = 32 * h + 4 * k < b.npad ? __ldcg(src + k) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            v[4 * k] += w[k].x;
+                            v[4 * k + 1] += w[k].y;
+                            v[4 * k + 2] += w[k].z;
+                            v[4 * k + 3] += w[k].w;
+                        }
                     }
                     if (r < pr.R) {
 #pragma unroll
