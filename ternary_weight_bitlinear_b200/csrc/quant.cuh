@@ -414,6 +414,7 @@ __global__ void __launch_bounds__(32 * W, MINB) quant_row_kernel(const __grid_co
     const uint4* xv = reinterpret_cast<const uint4*>(pr.x + (int64_t)m * pr.K);
     const uint4* gv = reinterpret_cast<const uint4*>(pr.gain);
     const bool norm = pr.gain != nullptr;
+    const int nv = (nvec + NTR - 1) / NTR;  // vector slots holding part of the row (same for all threads)
 
     float h[VPT][8];
     {
@@ -424,7 +425,8 @@ __global__ void __launch_bounds__(32 * W, MINB) quant_row_kernel(const __grid_co
             xr[i] = v < nvec ? __ldcg(xv + v) : make_uint4(0u, 0u, 0u, 0u);  // zeros add nothing
         }
 #pragma unroll
-        for (int i = 0; i < VPT; ++i) unpack8_bf16(xr[i], h[i]);
+        for (int i = 0; i < VPT; ++i)
+            if (i < nv) unpack8_bf16(xr[i], h[i]);
     }
 
     // reductions over the row's threads: shuffle tree, then warps in index order
@@ -481,12 +483,14 @@ __global__ void __launch_bounds__(32 * W, MINB) quant_row_kernel(const __grid_co
     if (norm) {
         double ss0 = 0.0, ss1 = 0.0;  // binary64 sums of the exact squares
 #pragma unroll
-        for (int i = 0; i < VPT; ++i)
+        for (int i = 0; i < VPT; ++i) {
+            if (i >= nv) break;  // slots past the row hold zeros for every thread
 #pragma unroll
             for (int j = 0; j < 8; j += 2) {
                 ss0 = __fma_rn((double)h[i][j], (double)h[i][j], ss0);
                 ss1 = __fma_rn((double)h[i][j + 1], (double)h[i][j + 1], ss1);
             }
+        }
         float r;
         if (!rms_factor_bounded(row_sum_d(__dadd_rn(ss0, ss1)), pr.K, b.eps, r)) {
             // rare: the interval straddles a rounding boundary; take the sum
@@ -520,9 +524,11 @@ __global__ void __launch_bounds__(32 * W, MINB) quant_row_kernel(const __grid_co
         }
     } else {
 #pragma unroll
-        for (int i = 0; i < VPT; ++i)
+        for (int i = 0; i < VPT; ++i) {
+            if (i >= nv) break;
 #pragma unroll
             for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(h[i][j]));
+        }
     }
     const float s = __fdiv_rn(127.0f, fmaxf(row_max(mx), kScaleFloor));
 
