@@ -10,8 +10,14 @@
 // the interval give the same binary32 value, else (rarely) the sum is redone
 // with error-free TwoSum accumulation.
 //
-// One CTA works on one token row; all loads are 16-byte vectors (8 bf16).  The
-// row is read from global memory once and staged in shared memory.
+// Kernels (all loads 16-byte vectors of 8 bf16, each row read from global
+// memory once):
+//   quant_batch_kernel  one CTA per row, staged in shared memory: few rows
+//                       (decode), lowest latency;
+//   quant_warp_kernel   one warp per row, staged in shared memory: many rows
+//                       longer than the register kernels hold;
+//   quant_row_kernel    one CTA of W warps per row, the row in registers:
+//                       many rows (prefill, batched decode).
 #pragma once
 
 #include "common.cuh"
