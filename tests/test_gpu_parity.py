@@ -116,6 +116,29 @@ def test_act_quant_matches_oracle(M, K, norm):
     assert_exact(rs.cpu().numpy(), rs_o, "row sums")
 
 
+@pytest.mark.parametrize("M,K", [(3, 256), (1024, 2560), (1030, 6912), (1024, 8208)])
+def test_act_quant_tie_rows(M, K):
+    """Rows with max|x| = 127 (scale exactly 1) and half-integer entries: every
+    quantiser kernel rounds the ties to the even neighbour, as the oracle."""
+    ties = [127.0, 0.5, 1.5, 2.5, 3.5, -0.5, -1.5, -2.5, 126.5, -126.5, 4.5, -3.5]
+    codes = [127, 0, 2, 2, 4, 0, -2, -2, 126, -126, 4, -4]
+    x = WL.activations(M, K, seed=M + 3 * K)
+    at = np.linspace(0, M - 1, min(M, 6)).astype(int)
+    row = np.zeros(K, np.float32)
+    row[:len(ties)] = ties
+    for i, m in enumerate(at):
+        x[m] = WL.to_bf16_bits(row if i % 2 == 0 else -row)
+    q, s, rs = B.bitlinear_act_quant(bf16_dev(x))
+    q_o, s_o, rs_o = O.quantize_input(x)
+    qh = q.cpu().numpy()
+    for i, m in enumerate(at):
+        sign = 1 if i % 2 == 0 else -1
+        assert list(qh[m, :len(codes)]) == [sign * c for c in codes]
+    assert_exact(s.cpu().numpy().view(np.uint32), s_o.view(np.uint32), "s_x")
+    assert_exact(qh, q_o, "codes")
+    assert_exact(rs.cpu().numpy(), rs_o, "row sums")
+
+
 @pytest.mark.parametrize("M,K", [(8, 2560),      # one CTA per row
                                  (1024, 2560),   # many rows: two warps per row
                                  (1031, 6912),   # four warps per row

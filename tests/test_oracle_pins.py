@@ -273,6 +273,23 @@ def test_act_quant_invariants(O):
     assert (err[big] <= (0.5 / s[big, None].astype(np.float64)) * (1 + 1e-6)).all()
 
 
+TIE_VALUES = [127.0, 0.5, 1.5, 2.5, 3.5, -0.5, -1.5, -2.5, 126.5, -126.5, 4.5, -3.5]
+TIE_CODES = [127, 0, 2, 2, 4, 0, -2, -2, 126, -126, 4, -4]  # halves go to the even neighbour
+
+
+def test_act_quant_rounds_ties_to_even(O):
+    """With max|h| = 127 the scale is exactly 1, so h = k + 1/2 lands on a tie:
+    the codes are the even neighbours (round half to even, as torch.round)."""
+    h = np.zeros((2, 16), np.float32)
+    h[0, :len(TIE_VALUES)] = TIE_VALUES
+    h[1, :len(TIE_VALUES)] = [-v for v in TIE_VALUES]
+    q, s, rs = O.act_quant(h)
+    assert s[0] == s[1] == np.float32(1.0)
+    np.testing.assert_array_equal(q[0, :len(TIE_CODES)], TIE_CODES)
+    np.testing.assert_array_equal(q[1, :len(TIE_CODES)], [-c for c in TIE_CODES])
+    np.testing.assert_array_equal(rs, [sum(TIE_CODES), -sum(TIE_CODES)])
+
+
 # --------------------------------------------------------------------------
 # RMSNorm
 # --------------------------------------------------------------------------
