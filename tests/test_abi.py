@@ -142,6 +142,38 @@ def test_batch_argument_checks(L):
     assert L.bitlinear_forward_batch(arr, 7, 0, 1e-5, NULL, 0, NULL) == 0  # M = 0: no-op
 
 
+def _qbatch(n, K=256, N=128, q=P16, rowsum=P16, dt=0, residual=None):
+    arr = (B.bitlinear.QuantizedProblem * n)()
+    for i in range(n):
+        arr[i] = B.bitlinear.QuantizedProblem(q.value if q else None, P16.value,
+                                              rowsum.value if rowsum else None, P16.value,
+                                              P16.value, residual.value if residual else None,
+                                              K, N, 1.0, dt)
+    return arr
+
+
+def test_quantized_batch_argument_checks(L):
+    Q = L.bitlinear_forward_quantized_batch
+    assert Q(NULL, 1, 8, NULL, 0, NULL) == 1
+    assert Q(_qbatch(1), 0, 8, NULL, 0, NULL) == 2                # count 0
+    assert Q(_qbatch(257), 257, 8, NULL, 0, NULL) == 2            # > BL_MAX_BATCH
+    assert Q(_qbatch(2), 2, -1, NULL, 0, NULL) == 2               # M < 0
+    assert Q(_qbatch(2, K=250), 2, 8, NULL, 0, NULL) == 2         # K % 16
+    assert Q(_qbatch(2, N=130), 2, 8, NULL, 0, NULL) == 2         # N % 4
+    assert Q(_qbatch(2, dt=5), 2, 8, NULL, 0, NULL) == 4          # unknown dtype
+    assert Q(_qbatch(2, dt=1, residual=P16), 2, 8, NULL, 0, NULL) == 4  # residual wants bf16
+    assert Q(_qbatch(2, q=None), 2, 8, NULL, 0, NULL) == 1
+    assert Q(_qbatch(2, rowsum=None), 2, 8, NULL, 0, NULL) == 1
+    assert Q(_qbatch(2, q=P17), 2, 8, NULL, 0, NULL) == 3
+    assert Q(_qbatch(2, q=None), 2, 0, NULL, 0, NULL) == 0        # M = 0: no-op, pointers unread
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_selftest_and_quantized_batch_need_a_device(L):
+    assert L.bitlinear_selftest_wait_timeout(1000000, NULL) == 8
+    assert L.bitlinear_forward_quantized_batch(_qbatch(2), 2, 8, NULL, 0, NULL) == 8
+
+
 def test_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 256, dtype=torch.bfloat16)
     P = torch.zeros(32, 256, dtype=torch.uint8)
