@@ -339,6 +339,27 @@ def test_rmsnorm_matches_textbook_formula(O):
     np.testing.assert_allclose(h, ref, rtol=4 * 2.0 ** -24, atol=0)
 
 
+def test_rescale_is_two_correctly_rounded_steps(O):
+    """y = RN32(RN32(acc * beta) / s_x), each step the correctly rounded value
+    of the exact rational (multiply first, then divide); the other order
+    differs on most of these samples."""
+    rng = np.random.default_rng(5)
+    M, N = 8, 64
+    acc = rng.integers(-877824, 877825, (M, N)).astype(np.int32)  # |acc| <= 127 * 6912
+    acc[0, :4] = [0, 1, -1, 877824]
+    s = (np.float32(127) / rng.uniform(0.5, 40, M).astype(np.float32)).astype(np.float32)
+    beta = np.float32(0.0173)
+    y = O.rescale(acc, s, float(beta))
+    swapped = 0
+    for m in range(M):
+        for n in range(N):
+            p = rn32_of_fraction(Fraction(int(acc[m, n])) * Fraction(float(beta)))
+            assert y[m, n] == rn32_of_fraction(Fraction(float(p)) / Fraction(float(s[m])))
+            d = rn32_of_fraction(Fraction(int(acc[m, n])) / Fraction(float(s[m])))
+            swapped += rn32_of_fraction(Fraction(float(d)) * Fraction(float(beta))) != y[m, n]
+    assert swapped > 0
+
+
 # --------------------------------------------------------------------------
 # Forward vs brute force
 # --------------------------------------------------------------------------
