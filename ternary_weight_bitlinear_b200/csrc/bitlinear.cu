@@ -195,8 +195,9 @@ bl_status launch_quant_cap(const QuantProblem* probs, int count, int64_t M, floa
         return launch(fn, dim3((unsigned)rows), dim3(32 * kQuantRowW2), 0, stream, b);
     }
     if (kmax <= kQuantWarpMaxK && rows >= kQuantWarpMinRows) {
-        // many rows (prefill): one warp per row, up to 8 rows per CTA; few rows
-        // (decode) go to one CTA per row below, which has the lower latency
+        // many rows longer than the register kernels hold: one warp per row
+        // staged in shared memory, up to 8 rows per CTA; few rows (decode) go
+        // to one CTA per row below, which has the lower latency
         const int wpb = (int)std::max<int64_t>(1, std::min<int64_t>(8, 65536 / (4 * (int64_t)kmax)));
         auto fn = quant_warp_kernel<CAP>;
         const int64_t smem = (int64_t)wpb * 4 * kmax;
