@@ -348,6 +348,41 @@ def test_batch_config2_layer(layer):
     _check_batch(items, refs, "config 2 layer %d batch" % layer)
 
 
+def test_batch_whole_token_as_timed():
+    """The timed decode step: all 210 projections of one token (30 layers) in one
+    batched call.  The GPU computes all of them; the oracle recomputes three
+    layers' seven outputs each (those layers with their seeded master weights,
+    the others with seeded weights drawn on the device)."""
+    items, check = [], {}
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(210)
+    for layer in range(WL.LAYERS):
+        for p in WL.PROJECTIONS:
+            c = WL.config2_projection(layer, p.name)
+            if layer in (0, 14, 29):
+                W = WL.master_weights(p.N, p.K, WL.master_seed(layer, p.name))
+                W_d = torch.from_numpy(W).cuda()
+            else:
+                W = None
+                W_d = torch.randn(p.N, p.K, device="cuda", generator=gen) * WL.MASTER_STD
+            P_d, beta_d = B.bitlinear_pack(W_d)
+            del W_d
+            items.append(dict(x=bf16_dev(c["x"]), gain=bf16_dev(c["gain"]), P=P_d,
+                              beta=float(beta_d.item()),
+                              y=torch.empty((1, p.N), dtype=torch.bfloat16, device="cuda")))
+            if W is not None:
+                check[len(items) - 1] = (c, W)
+    assert len(items) == 210
+    B.bitlinear_forward_batch(B.make_batch(items), 1, WL.RMS_EPS)
+    for i, (c, W) in check.items():
+        P_o, beta_o = O.pack_master(W)
+        assert np.float32(items[i]["beta"]) == np.float32(beta_o)
+        assert_exact(items[i]["P"].cpu().numpy(), P_o, "packed bytes %d" % i)
+        ref = O.f32_to_bf16(O.forward(c["x"], P_o, beta_o, gain=c["gain"], eps=WL.RMS_EPS,
+                                      norm=True)["y"])
+        assert_bf16_output(bf16_host(items[i]["y"]), ref, "token batch problem %d" % i)
+
+
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5])
 def test_batch_mixed_problems(M):
     specs = [(256, 128, True, torch.bfloat16, False), (2560, 640, False, torch.float32, False),
