@@ -230,19 +230,23 @@ bl_status bitlinear_accumulate(const int8_t* q, const int32_t* rowsum, const uin
 #define BL_NOALLOC_SCRATCH_BYTES (2u << 20)
 
 /* Same computation and result as bitlinear_forward, for callers that cannot
- * allocate device memory: code running while a CUDA graph is being captured
- * (cudaMalloc is not allowed there), latency-critical loops that must not pay
+ * allocate device memory: latency-critical loops that must not pay
  * cudaMalloc/cudaFree's implicit device synchronisation, and plugins embedded
- * in an engine that owns every allocation itself.  (The method's own pages
- * have no counterpart; this is an interface convenience.)
+ * in an engine that owns every allocation itself and hands them only their
+ * inputs and outputs.  (The method's own pages have no counterpart; this is an
+ * interface convenience.)
  *   Arguments as in bitlinear_forward, without the workspace.
  *   Scratch: instead of a caller workspace it uses one file-scope device array
  *   of BL_NOALLOC_SCRATCH_BYTES that every GPU which loads the library keeps
  *   until the process exits.  The first call on a device looks up that array's
  *   device address (so make that first call before any stream capture).
- *   Shapes whose workspace (bitlinear_forward_workspace_size) exceeds the
- *   array are rejected with BL_ERR_WORKSPACE before anything is launched, and
- *   bitlinear_last_error() names both sizes.
+ *   The array must hold the int8 codes, scales and row sums of the input
+ *   (M*K bytes plus 8*M, each part rounded up to 256 bytes); larger shapes are
+ *   rejected with BL_ERR_WORKSPACE before anything is launched, and
+ *   bitlinear_last_error() names both sizes.  For 5 <= M <= 64, when the
+ *   split-tile tail of bitlinear_forward_workspace_size does not fit beside
+ *   the codes, the CTA shares are cut at row-tile boundaries instead (same
+ *   results).
  *   All calls share the one array: calls that can overlap on the GPU (other
  *   streams, other host threads) race on it and must be serialised by the
  *   caller.  Nothing in it needs to start at zero: every byte a call reads was

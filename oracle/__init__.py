@@ -11,7 +11,7 @@ passed as ``numpy.uint16`` arrays holding the bf16 bit patterns.
 Function          Definition followed
 ----------------  ----------------------------------------------------------
 weight_scale      absmean of |W| clamped at 1e-5 (the per-tensor weight scale)
-ternarize         clamp(round(W / beta), -1, 1)
+ternarize         clamp(round(W * RN32(1/beta)), -1, 1): multiply by the scale
 pack / unpack     2-bit codes t+1, four rows per byte, bit pair i = quarter i
 rmsnorm           exact-sum RMSNorm, gain after the rms factor
 act_quant         per-token absmax int8: s = 127/max(max|h|,1e-5), round, clamp

@@ -611,10 +611,18 @@ bl_status bitlinear_forward_workspace_size(int64_t M, int64_t K, int64_t N, size
     return BL_OK;
 }
 
-bl_status bitlinear_forward(const uint16_t* x, const uint16_t* gain, float eps, const uint8_t* P,
-                            float beta, int64_t M, int64_t K, int64_t N, void* y,
-                            bl_out_dtype y_dtype, void* workspace, size_t workspace_bytes,
-                            void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The forward behind bitlinear_forward and bitlinear_forward_noalloc.  The
+// workspace holds the codes, scales and row sums (ws_problem_bytes) and, when
+// `need_split` (or when it is large enough anyway), the split-tile tail of the
+// 5..64-token kernel; without that tail the kernel cuts its CTA shares at
+// row-tile boundaries, with the same results.
+bl_status forward_impl(const uint16_t* x, const uint16_t* gain, float eps, const uint8_t* P,
+                       float beta, int64_t M, int64_t K, int64_t N, void* y, bl_out_dtype y_dtype,
+                       void* workspace, size_t workspace_bytes, bool need_split, void* stream) {
     bl_status st = check_shape(M, K, N);
     if (st != BL_OK) return st;
     const int epi = epi_of(y_dtype);
@@ -624,7 +632,8 @@ bl_status bitlinear_forward(const uint16_t* x, const uint16_t* gain, float eps, 
     if (!aligned16(x) || !aligned16(P) || !aligned16(y) || (gain && !aligned16(gain)))
         return BL_ERR_ALIGN;
     const int64_t own = ws_problem_bytes(M, K);
-    if (!workspace || workspace_bytes < (size_t)(own + sk_ws_bytes(M))) return BL_ERR_WORKSPACE;
+    const int64_t need = own + (need_split ? sk_ws_bytes(M) : 0);
+    if (!workspace || workspace_bytes < (size_t)need) return BL_ERR_WORKSPACE;
     if (!aligned16(workspace)) return BL_ERR_ALIGN;
     int dev;
     DeviceInfo info;
@@ -635,7 +644,19 @@ bl_status bitlinear_forward(const uint16_t* x, const uint16_t* gain, float eps, 
     QuantProblem qp = {x, gain, w.q, w.s_x, w.rowsum, (int)K};
     if ((st = run_quant(&qp, 1, M, eps, dev, info, s)) != BL_OK) return st;
     return run_quantized(w.q, w.s_x, w.rowsum, P, beta, M, K, N, y, epi, nullptr, dev, info, s,
-                         static_cast<char*>(workspace) + own, (size_t)sk_ws_bytes(M));
+                         static_cast<char*>(workspace) + own, workspace_bytes - (size_t)own);
+}
+
+}  // namespace
+
+extern "C" {
+
+bl_status bitlinear_forward(const uint16_t* x, const uint16_t* gain, float eps, const uint8_t* P,
+                            float beta, int64_t M, int64_t K, int64_t N, void* y,
+                            bl_out_dtype y_dtype, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+    return forward_impl(x, gain, eps, P, beta, M, K, N, y, y_dtype, workspace, workspace_bytes,
+                        true, stream);
 }
 
 bl_status bitlinear_forward_batch_workspace_size(const bl_problem* probs, int count, int64_t M,
@@ -826,14 +847,16 @@ bl_status bitlinear_selftest_wait_timeout(int64_t limit_ns, void* stream) {
 bl_status bitlinear_forward_noalloc(const uint16_t* x, const uint16_t* gain, float eps,
                                     const uint8_t* P, float beta, int64_t M, int64_t K,
                                     int64_t N, void* y, bl_out_dtype y_dtype, void* stream) {
-    size_t need = 0;
-    bl_status st = bitlinear_forward_workspace_size(M, K, N, &need);
+    bl_status st = check_shape(M, K, N);
     if (st != BL_OK) return st;
-    if (need > BL_NOALLOC_SCRATCH_BYTES) {
+    // the scratch must hold the codes, scales and row sums; the split-tile
+    // tail of the 5..64-token kernel is used only when it fits as well
+    const int64_t need = M == 0 ? 0 : ws_problem_bytes(M, K);
+    if (need > (int64_t)BL_NOALLOC_SCRATCH_BYTES) {
         snprintf(g_last_error, sizeof g_last_error,
-                 "bitlinear_forward_noalloc: this shape needs %zu bytes of scratch; the fixed "
+                 "bitlinear_forward_noalloc: this shape needs %lld bytes of scratch; the fixed "
                  "scratch holds %u",
-                 need, (unsigned)BL_NOALLOC_SCRATCH_BYTES);
+                 (long long)need, (unsigned)BL_NOALLOC_SCRATCH_BYTES);
         return BL_ERR_WORKSPACE;
     }
     void* scratch = nullptr;
@@ -843,8 +866,8 @@ bl_status bitlinear_forward_noalloc(const uint16_t* x, const uint16_t* gain, flo
         if ((st = current_device(&dev, &info)) != BL_OK) return st;
         if ((st = noalloc_scratch(dev, &scratch)) != BL_OK) return st;
     }
-    return bitlinear_forward(x, gain, eps, P, beta, M, K, N, y, y_dtype, scratch,
-                             need > 0 ? (size_t)BL_NOALLOC_SCRATCH_BYTES : 0, stream);
+    return forward_impl(x, gain, eps, P, beta, M, K, N, y, y_dtype, scratch,
+                        need > 0 ? (size_t)BL_NOALLOC_SCRATCH_BYTES : 0, false, stream);
 }
 
 }  // extern "C"

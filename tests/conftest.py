@@ -81,3 +81,12 @@ def O():
     import oracle
     oracle.lib()
     return oracle
+
+
+@pytest.fixture
+def guard():
+    """Guarded device buffers (see gpu_util.Guard); checked after the test."""
+    from gpu_util import Guard
+    g = Guard()
+    yield g
+    g.check()

@@ -63,3 +63,52 @@ def assert_exact(got, ref, what=""):
     assert bad.size == 0, "%s: %d of %d differ (first at %s: %r vs %r)" % (
         what, bad.size, got.size, np.unravel_index(bad[0], got.shape), got.flat[bad[0]],
         ref.flat[bad[0]])
+
+
+# ---------------------------------------------------------------------------
+# guard canaries: out-of-bounds writes show up as changed pattern bytes
+# ---------------------------------------------------------------------------
+GUARD_BYTES = 4096
+GUARD_FILL = 0xA5
+
+
+class Guard:
+    """Hands out device buffers that sit between two GUARD_BYTES-long runs of
+    the byte GUARD_FILL inside one allocation.  ``check()`` asserts that every
+    run is unchanged, so a kernel that writes past either end of an output or
+    a workspace fails the test even when the values it was asked for are
+    right.  The buffer itself starts GUARD_BYTES into the allocation, so its
+    alignment is the allocation's (256 bytes) whatever its size."""
+
+    def __init__(self):
+        self.bufs = []
+
+    def empty(self, shape, dtype, fill=None):
+        shape = tuple(shape) if isinstance(shape, (tuple, list)) else (shape,)
+        n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        raw = torch.full((2 * GUARD_BYTES + n,), GUARD_FILL, dtype=torch.uint8, device="cuda")
+        body = raw[GUARD_BYTES:GUARD_BYTES + n]
+        if fill is not None:
+            body.fill_(fill)
+        self.bufs.append((raw, n, "%s %s" % (shape, dtype)))
+        return body.view(dtype).view(shape)
+
+    def copy(self, t):
+        """A guarded copy of a CUDA tensor (inputs updated in place, residuals)."""
+        g = self.empty(t.shape, t.dtype)
+        g.copy_(t)
+        return g
+
+    def workspace(self, nbytes):
+        """A guarded uint8 workspace of exactly nbytes (None when 0)."""
+        return self.empty((nbytes,), torch.uint8) if nbytes else None
+
+    def check(self):
+        torch.cuda.synchronize()
+        for raw, n, what in self.bufs:
+            lo = raw[:GUARD_BYTES].cpu().numpy()
+            hi = raw[GUARD_BYTES + n:].cpu().numpy()
+            for side, run in (("before", lo), ("after", hi)):
+                bad = np.flatnonzero(run != GUARD_FILL)
+                assert bad.size == 0, "guard bytes %s the buffer %s were overwritten (%d bytes, " \
+                    "first at offset %d)" % (side, what, bad.size, int(bad[0]))

@@ -33,12 +33,17 @@ def both_pack(W):
     return P_d, beta_g, P_o, beta_o
 
 
-def run_forward(cfg, P_d, beta, P_o, beta_o, what):
+def run_forward(cfg, P_d, beta, P_o, beta_o, what, guard):
+    """Forward through the C ABI into a guarded output and an exactly sized
+    guarded workspace, checked against the oracle."""
     x = cfg["x"]
     gain = cfg.get("gain") if cfg["norm"] else None
     out_dtype = torch.float32 if cfg["out"] == "f32" else torch.bfloat16
+    M, K = x.shape
+    N = 4 * P_d.shape[0]
     y = B.bitlinear_forward(bf16_dev(x), P_d, beta, gain=None if gain is None else bf16_dev(gain),
-                            eps=WL.RMS_EPS, out_dtype=out_dtype)
+                            eps=WL.RMS_EPS, out=guard.empty((M, N), out_dtype),
+                            workspace=guard.workspace(B.bitlinear_forward_workspace_size(M, K, N)))
     ref = O.forward(x, P_o, beta_o, gain=gain, eps=WL.RMS_EPS, norm=cfg["norm"])
     if out_dtype == torch.float32:
         assert_f32_output(y.cpu().numpy(), ref["y"], what)
@@ -105,11 +110,17 @@ def special_rows(x):
                                  # shared-memory warp kernel
                                  (1024, 2560), (1031, 6912), (1100, 272), (1024, 2576),
                                  (1025, 7168), (1024, 8192), (1030, 8208)])
-def test_act_quant_matches_oracle(M, K, norm):
+def guarded_quant(guard, M, K):
+    """Guarded code, scale and row-sum buffers for an [M,K] quantisation."""
+    return dict(q=guard.empty((M, K), torch.int8), s_x=guard.empty(M, torch.float32),
+                rowsum=guard.empty(M, torch.int32))
+
+
+def test_act_quant_matches_oracle(M, K, norm, guard):
     x = special_rows(WL.activations(M, K, seed=M * 131 + K, outlier_frac=0.001))
     gain = WL.gain(K, seed=K) if norm else None
     q, s, rs = B.bitlinear_act_quant(bf16_dev(x), None if gain is None else bf16_dev(gain),
-                                     WL.RMS_EPS)
+                                     WL.RMS_EPS, **guarded_quant(guard, M, K))
     q_o, s_o, rs_o = O.quantize_input(x, gain, WL.RMS_EPS, norm=norm)
     assert_exact(s.cpu().numpy().view(np.uint32), s_o.view(np.uint32), "s_x")
     assert_exact(q.cpu().numpy(), q_o, "codes")
@@ -117,7 +128,7 @@ def test_act_quant_matches_oracle(M, K, norm):
 
 
 @pytest.mark.parametrize("M,K", [(3, 256), (1024, 2560), (1030, 6912), (1024, 8208)])
-def test_act_quant_tie_rows(M, K):
+def test_act_quant_tie_rows(M, K, guard):
     """Rows with max|x| = 127 (scale exactly 1) and half-integer entries: every
     quantiser kernel rounds the ties to the even neighbour, as the oracle."""
     ties = [127.0, 0.5, 1.5, 2.5, 3.5, -0.5, -1.5, -2.5, 126.5, -126.5, 4.5, -3.5]
@@ -128,7 +139,7 @@ def test_act_quant_tie_rows(M, K):
     row[:len(ties)] = ties
     for i, m in enumerate(at):
         x[m] = WL.to_bf16_bits(row if i % 2 == 0 else -row)
-    q, s, rs = B.bitlinear_act_quant(bf16_dev(x))
+    q, s, rs = B.bitlinear_act_quant(bf16_dev(x), **guarded_quant(guard, M, K))
     q_o, s_o, rs_o = O.quantize_input(x)
     qh = q.cpu().numpy()
     for i, m in enumerate(at):
@@ -144,7 +155,7 @@ def test_act_quant_tie_rows(M, K):
                                  (1031, 6912),   # four warps per row
                                  (1024, 8208),   # past 7168: the shared-memory warp kernel
                                  (1, 16)])
-def test_act_quant_rms_boundary_rows(M, K):
+def test_act_quant_rms_boundary_rows(M, K, guard):
     """Rows whose RMSNorm factor is decided by the rounding of the exact sum of
     squares (the fast interval test must fall back to the exact sum) at
     several places of the batch."""
@@ -154,7 +165,8 @@ def test_act_quant_rms_boundary_rows(M, K):
     at = np.linspace(0, M - 1, n).astype(int)
     x[at] = straddle_rows(n, K, WL.RMS_EPS, seed=K + M)
     gain = WL.gain(K, seed=K + 1)
-    q, s, rs = B.bitlinear_act_quant(bf16_dev(x), bf16_dev(gain), WL.RMS_EPS)
+    q, s, rs = B.bitlinear_act_quant(bf16_dev(x), bf16_dev(gain), WL.RMS_EPS,
+                                     **guarded_quant(guard, M, K))
     q_o, s_o, rs_o = O.quantize_input(x, gain, WL.RMS_EPS, norm=True)
     assert_exact(s.cpu().numpy().view(np.uint32), s_o.view(np.uint32), "s_x")
     assert_exact(q.cpu().numpy(), q_o, "codes")
@@ -166,14 +178,14 @@ def test_act_quant_rms_boundary_rows(M, K):
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("M,K,N", [(1, 16, 4), (2, 64, 12), (3, 256, 128), (4, 2560, 640),
                                    (5, 272, 36), (9, 6912, 2560), (1, 65536, 8), (2, 65536, 8)])
-def test_accumulate_is_exact(M, K, N):
+def test_accumulate_is_exact(M, K, N, guard):
     x = special_rows(WL.activations(M, K, seed=M + K + N, row_std=(0.1, 10.0)))
     W = WL.master_weights(N, K, seed=K + N)
     P_d, beta, P_o, beta_o = both_pack(W)
     q, s, rs = B.bitlinear_act_quant(bf16_dev(x))
     q_o, s_o, rs_o = O.quantize_input(x)
     assert_exact(q.cpu().numpy(), q_o, "codes")
-    acc = B.bitlinear_accumulate(q, rs, P_d)
+    acc = B.bitlinear_accumulate(q, rs, P_d, out=guard.empty((M, N), torch.int32))
     acc_o = O.ternary_matmul(q_o, O.unpack(P_o))
     assert_exact(acc.cpu().numpy(), acc_o, "int32 accumulators")
 
@@ -181,33 +193,33 @@ def test_accumulate_is_exact(M, K, N):
 # ---------------------------------------------------------------------------
 # the five workloads
 # ---------------------------------------------------------------------------
-def test_config1_single_bitlinear_fp32():
+def test_config1_single_bitlinear_fp32(guard):
     c = WL.config1()
     P_d, beta, P_o, beta_o = both_pack(c["W"])
-    y, ref = run_forward(c, P_d, beta, P_o, beta_o, "config 1")
+    y, ref = run_forward(c, P_d, beta, P_o, beta_o, "config 1", guard)
     assert not y[1].any()                      # the all-zero token gives +0 outputs
     assert not torch.signbit(y[1]).any()
 
 
 @pytest.mark.parametrize("layer", [0, 29])
-def test_config2_decode_all_projections(layer):
+def test_config2_decode_all_projections(layer, guard):
     for p in WL.PROJECTIONS:
         c = WL.config2_projection(layer, p.name)
         W = WL.master_weights(p.N, p.K, WL.master_seed(layer, p.name))
         P_d, beta, P_o, beta_o = both_pack(W)
-        run_forward(c, P_d, beta, P_o, beta_o, "config 2 %s" % p.name)
+        run_forward(c, P_d, beta, P_o, beta_o, "config 2 %s" % p.name, guard)
 
 
 @pytest.mark.parametrize("M", [8, 32, 64])
-def test_config3_batched_decode(M):
+def test_config3_batched_decode(M, guard):
     for p in WL.PROJECTIONS:
         c = WL.config3_projection(0, p.name, M)
         W = WL.master_weights(p.N, p.K, WL.master_seed(0, p.name))
         P_d, beta, P_o, beta_o = both_pack(W)
-        run_forward(c, P_d, beta, P_o, beta_o, "config 3 %s M=%d" % (p.name, M))
+        run_forward(c, P_d, beta, P_o, beta_o, "config 3 %s M=%d" % (p.name, M), guard)
 
 
-def test_config4_prefill_sampled_rows():
+def test_config4_prefill_sampled_rows(guard):
     """M=4096: the GPU computes every row; the oracle recomputes a sample of
     rows (rows are independent) and the full int8 codes of one projection."""
     rng = np.random.default_rng(4096)
@@ -217,7 +229,10 @@ def test_config4_prefill_sampled_rows():
         W = WL.master_weights(p.N, p.K, WL.master_seed(0, name))
         P_d, beta, P_o, beta_o = both_pack(W)
         x_d, g_d = bf16_dev(c["x"]), bf16_dev(c["gain"])
-        y = bf16_host(B.bitlinear_forward(x_d, P_d, beta, gain=g_d, eps=WL.RMS_EPS))
+        M = c["x"].shape[0]
+        y = bf16_host(B.bitlinear_forward(
+            x_d, P_d, beta, gain=g_d, eps=WL.RMS_EPS, out=guard.empty((M, p.N), torch.bfloat16),
+            workspace=guard.workspace(B.bitlinear_forward_workspace_size(M, p.K, p.N))))
         rows = np.unique(np.concatenate([[0, 1, 4095], rng.integers(0, 4096, 29)]))
         ref = O.forward(c["x"][rows], P_o, beta_o, gain=c["gain"], eps=WL.RMS_EPS, norm=True)
         assert_bf16_output(y[rows], O.f32_to_bf16(ref["y"]), "config 4 %s" % name)
@@ -228,28 +243,32 @@ def test_config4_prefill_sampled_rows():
             assert_exact(s.cpu().numpy().view(np.uint32), s_o.view(np.uint32), "config 4 s_x")
 
 
-def gpu_ffn_block(x_d, g_in, g_sub, Pg, bg, Pu, bu, Pd, bd):
-    """One FFN block through the C ABI; updates x_d in place."""
-    q, s, rs = B.bitlinear_act_quant(x_d, g_in, WL.RMS_EPS)
-    a = B.bitlinear_forward_quantized(q, s, rs, Pg, bg)
-    b = B.bitlinear_forward_quantized(q, s, rs, Pu, bu)
-    z = B.bitlinear_relu2_mul(a, b)
-    q2, s2, rs2 = B.bitlinear_act_quant(z, g_sub, WL.RMS_EPS)
+def gpu_ffn_block(x_d, g_in, g_sub, Pg, bg, Pu, bu, Pd, bd, guard):
+    """One FFN block through the C ABI, every intermediate in a guarded
+    buffer; updates x_d in place."""
+    M, H = x_d.shape
+    I = 4 * Pg.shape[0]
+    q, s, rs = B.bitlinear_act_quant(x_d, g_in, WL.RMS_EPS, **guarded_quant(guard, M, H))
+    a = B.bitlinear_forward_quantized(q, s, rs, Pg, bg, out=guard.empty((M, I), torch.bfloat16))
+    b = B.bitlinear_forward_quantized(q, s, rs, Pu, bu, out=guard.empty((M, I), torch.bfloat16))
+    z = B.bitlinear_relu2_mul(a, b, out=guard.empty((M, I), torch.bfloat16))
+    q2, s2, rs2 = B.bitlinear_act_quant(z, g_sub, WL.RMS_EPS, **guarded_quant(guard, M, I))
     B.bitlinear_forward_quantized(q2, s2, rs2, Pd, bd, residual=x_d, out=x_d)
     return x_d
 
 
-def test_config5_ffn_chain_30_layers():
+def test_config5_ffn_chain_30_layers(guard):
     M = 16
     x = WL.config5_input(M)
-    x_d = bf16_dev(x)
+    x_d = guard.copy(bf16_dev(x))
     x_o = x.copy()
     for layer in range(WL.LAYERS):
         L = WL.config5_layer(layer)
         Pg, bg, Pg_o, bg_o = both_pack(L["W_gate"])
         Pu, bu, Pu_o, bu_o = both_pack(L["W_up"])
         Pd, bd, Pd_o, bd_o = both_pack(L["W_down"])
-        gpu_ffn_block(x_d, bf16_dev(L["g_in"]), bf16_dev(L["g_sub"]), Pg, bg, Pu, bu, Pd, bd)
+        gpu_ffn_block(x_d, bf16_dev(L["g_in"]), bf16_dev(L["g_sub"]), Pg, bg, Pu, bu, Pd, bd,
+                      guard)
         x_o = O.ffn_block(x_o, L["g_in"], L["g_sub"], WL.RMS_EPS, Pg_o, bg_o, Pu_o, bu_o, Pd_o,
                           bd_o)
         assert_bf16_output(bf16_host(x_d), x_o, "config 5 after layer %d" % layer)
@@ -259,22 +278,22 @@ def test_config5_ffn_chain_30_layers():
 # glue and edge cases
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("n", [8, 13, 6912 * 16, 1000003])
-def test_relu2_mul_matches_oracle(n):
+def test_relu2_mul_matches_oracle(n, guard):
     rng = np.random.default_rng(n)
     a = WL.to_bf16_bits((rng.standard_normal(n) * 3).astype(np.float32))
     b = WL.to_bf16_bits((rng.standard_normal(n) * 3).astype(np.float32))
-    z = B.bitlinear_relu2_mul(bf16_dev(a), bf16_dev(b))
+    z = B.bitlinear_relu2_mul(bf16_dev(a), bf16_dev(b), out=guard.empty(n, torch.bfloat16))
     assert_exact(bf16_host(z), O.relu2_mul(a, b), "relu2_mul")
 
 
-def test_residual_epilogue_matches_oracle():
+def test_residual_epilogue_matches_oracle(guard):
     M, K, N = 6, 256, 64
     x = WL.activations(M, K, seed=77)
     res = WL.activations(M, N, seed=78)
     W = WL.master_weights(N, K, seed=79)
     P_d, beta, P_o, beta_o = both_pack(W)
     q, s, rs = B.bitlinear_act_quant(bf16_dev(x))
-    r_d = bf16_dev(res)
+    r_d = guard.copy(bf16_dev(res))
     B.bitlinear_forward_quantized(q, s, rs, P_d, beta, residual=r_d, out=r_d)
     y_o = O.forward(x, P_o, beta_o)["y"]
     assert_exact(bf16_host(r_d), O.residual_add(res, O.f32_to_bf16(y_o)), "residual epilogue")
@@ -289,28 +308,30 @@ def test_empty_batch_is_a_no_op():
 
 @pytest.mark.parametrize("M,K,N", [(1, 16, 4), (2, 32, 8), (3, 4096 + 16, 12), (4, 16384, 20),
                                    (5, 64, 4), (1, 65536, 16), (3, 65536, 8)])
-def test_ragged_and_extreme_shapes(M, K, N):
+def test_ragged_and_extreme_shapes(M, K, N, guard):
     x = WL.activations(M, K, seed=M * K + N, outlier_frac=0.01)
     g = WL.gain(K, seed=N)
     W = WL.master_weights(N, K, seed=K - N)
     P_d, beta, P_o, beta_o = both_pack(W)
     for norm in (False, True):
         c = dict(x=x, gain=g, norm=norm, out="f32")
-        run_forward(c, P_d, beta, P_o, beta_o, "M=%d K=%d N=%d norm=%s" % (M, K, N, norm))
+        run_forward(c, P_d, beta, P_o, beta_o, "M=%d K=%d N=%d norm=%s" % (M, K, N, norm),
+                    guard)
 
 
 # ---------------------------------------------------------------------------
 # batched forwards (independent problems in one call)
 # ---------------------------------------------------------------------------
-def _batch_case(specs, M, seed):
-    """specs: list of (K, N, norm, out dtype, residual) -> (items, oracle outputs)."""
+def _batch_case(specs, M, seed, guard):
+    """specs: list of (K, N, norm, out dtype, residual) -> (items, oracle outputs);
+    outputs in guarded buffers."""
     items, refs = [], []
     for i, (K, N, norm, dt, res) in enumerate(specs):
         x = WL.activations(M, K, seed=seed + i, outlier_frac=0.001)
         g = WL.gain(K, seed=seed + 100 + i) if norm else None
         P_d, beta, P_o, beta_o = both_pack(WL.master_weights(N, K, seed=seed + 200 + i))
         y_o = O.forward(x, P_o, beta_o, gain=g, eps=WL.RMS_EPS, norm=norm)["y"]
-        it = dict(x=bf16_dev(x), P=P_d, beta=beta, y=torch.empty((M, N), dtype=dt, device="cuda"))
+        it = dict(x=bf16_dev(x), P=P_d, beta=beta, y=guard.empty((M, N), dt))
         if norm:
             it["gain"] = bf16_dev(g)
         if res:
@@ -325,6 +346,20 @@ def _batch_case(specs, M, seed):
     return items, refs
 
 
+def run_batch(items, M, guard):
+    """bitlinear_forward_batch with an exactly sized guarded workspace."""
+    arr = B.make_batch(items)
+    B.bitlinear_forward_batch(arr, M, WL.RMS_EPS,
+                              workspace=guard.workspace(B.bitlinear_forward_batch_workspace_size(arr, M)))
+
+
+def run_quantized_batch(items, M, guard):
+    """bitlinear_forward_quantized_batch with an exactly sized guarded workspace."""
+    B.bitlinear_forward_quantized_batch(
+        B.make_quantized_batch(items), M,
+        workspace=guard.workspace(B.bitlinear_quantized_batch_workspace_size(M)))
+
+
 def _check_batch(items, refs, what):
     for i, (it, (kind, ref)) in enumerate(zip(items, refs)):
         if kind == "f32":
@@ -334,7 +369,7 @@ def _check_batch(items, refs, what):
 
 
 @pytest.mark.parametrize("layer", [0, 17])
-def test_batch_config2_layer(layer):
+def test_batch_config2_layer(layer, guard):
     """A decode layer's seven projections (independent inputs) as one batch."""
     items, refs = [], []
     for p in WL.PROJECTIONS:
@@ -343,12 +378,12 @@ def test_batch_config2_layer(layer):
         refs.append(("bf16", O.f32_to_bf16(O.forward(c["x"], P_o, beta_o, gain=c["gain"],
                                                      eps=WL.RMS_EPS, norm=True)["y"])))
         items.append(dict(x=bf16_dev(c["x"]), gain=bf16_dev(c["gain"]), P=P_d, beta=beta,
-                          y=torch.empty((1, p.N), dtype=torch.bfloat16, device="cuda")))
-    B.bitlinear_forward_batch(B.make_batch(items), 1, WL.RMS_EPS)
+                          y=guard.empty((1, p.N), torch.bfloat16)))
+    run_batch(items, 1, guard)
     _check_batch(items, refs, "config 2 layer %d batch" % layer)
 
 
-def test_batch_whole_token_as_timed():
+def test_batch_whole_token_as_timed(guard):
     """The timed decode step: all 210 projections of one token (30 layers) in one
     batched call.  The GPU computes all of them; the oracle recomputes three
     layers' seven outputs each (those layers with their seeded master weights,
@@ -369,11 +404,11 @@ def test_batch_whole_token_as_timed():
             del W_d
             items.append(dict(x=bf16_dev(c["x"]), gain=bf16_dev(c["gain"]), P=P_d,
                               beta=float(beta_d.item()),
-                              y=torch.empty((1, p.N), dtype=torch.bfloat16, device="cuda")))
+                              y=guard.empty((1, p.N), torch.bfloat16)))
             if W is not None:
                 check[len(items) - 1] = (c, W)
     assert len(items) == 210
-    B.bitlinear_forward_batch(B.make_batch(items), 1, WL.RMS_EPS)
+    run_batch(items, 1, guard)
     for i, (c, W) in check.items():
         P_o, beta_o = O.pack_master(W)
         assert np.float32(items[i]["beta"]) == np.float32(beta_o)
@@ -384,24 +419,24 @@ def test_batch_whole_token_as_timed():
 
 
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5])
-def test_batch_mixed_problems(M):
+def test_batch_mixed_problems(M, guard):
     specs = [(256, 128, True, torch.bfloat16, False), (2560, 640, False, torch.float32, False),
              (6912, 2560, True, torch.bfloat16, True), (16, 4, False, torch.bfloat16, False),
              (4096 + 16, 12, True, torch.float32, False)]
-    items, refs = _batch_case(specs, M, seed=5000 + M)
-    B.bitlinear_forward_batch(B.make_batch(items), M, WL.RMS_EPS)
+    items, refs = _batch_case(specs, M, seed=5000 + M, guard=guard)
+    run_batch(items, M, guard)
     _check_batch(items, refs, "mixed batch M=%d" % M)
 
 
-def test_batch_many_problems():
+def test_batch_many_problems(guard):
     specs = [(16 * (1 + i % 7), 4 * (1 + i % 5), i % 2 == 0, torch.bfloat16, i % 3 == 0)
              for i in range(40)]
-    items, refs = _batch_case(specs, 2, seed=7000)
-    B.bitlinear_forward_batch(B.make_batch(items), 2, WL.RMS_EPS)
+    items, refs = _batch_case(specs, 2, seed=7000, guard=guard)
+    run_batch(items, 2, guard)
     _check_batch(items, refs, "40-problem batch")
 
 
-def test_quantized_batch_shared_input_qkv_and_gate_up():
+def test_quantized_batch_shared_input_qkv_and_gate_up(guard):
     """q|k|v share one quantised input, gate|up another: one launch each."""
     for M in (1, 3, 6):
         x = WL.activations(M, 2560, seed=8000 + M, outlier_frac=0.001)
@@ -416,19 +451,19 @@ def test_quantized_batch_shared_input_qkv_and_gate_up():
                 refs.append(O.f32_to_bf16(O.forward(x, P_o, beta_o, gain=g, eps=WL.RMS_EPS,
                                                     norm=True)["y"]))
                 items.append(dict(q=q, s_x=s, rowsum=rs, P=P_d, beta=beta,
-                                  y=torch.empty((M, p.N), dtype=torch.bfloat16, device="cuda")))
-            B.bitlinear_forward_quantized_batch(B.make_quantized_batch(items), M)
+                                  y=guard.empty((M, p.N), torch.bfloat16)))
+            run_quantized_batch(items, M, guard)
             for it, ref, name in zip(items, refs, names):
                 assert_bf16_output(bf16_host(it["y"]), ref, "shared-input %s M=%d" % (name, M))
 
 
-def test_batch_of_many_tiny_problems_and_one_large():
+def test_batch_of_many_tiny_problems_and_one_large(guard):
     """100 one-row problems land in the first CTA's byte range (more problems
     than a CTA stages), next to a large one: both code paths in one launch."""
     specs = [(16, 4, i % 2 == 0, torch.bfloat16, False) for i in range(100)]
     specs.append((2560, 2560, True, torch.float32, False))
-    items, refs = _batch_case(specs, 1, seed=9000)
-    B.bitlinear_forward_batch(B.make_batch(items), 1, WL.RMS_EPS)
+    items, refs = _batch_case(specs, 1, seed=9000, guard=guard)
+    run_batch(items, 1, guard)
     _check_batch(items, refs, "100 tiny + 1 large")
 
 
@@ -447,7 +482,7 @@ def test_batch_of_many_tiny_problems_and_one_large():
     (256, 144, 20384, "f32", False),   # R=5096: second half of the last tile 8 rows
     (200, 256, 20480, "i32", False),   # R=5120: every half full, int32 accumulators
 ])
-def test_gemm_path_shapes(M, K, N, out, residual):
+def test_gemm_path_shapes(M, K, N, out, residual, guard):
     x = special_rows(WL.activations(M, K, seed=M * 7 + K, row_std=(0.1, 10.0)))
     W = WL.master_weights(N, K, seed=N * 3 + K)
     P_d, beta, P_o, beta_o = both_pack(W)
@@ -455,16 +490,17 @@ def test_gemm_path_shapes(M, K, N, out, residual):
     q_o, s_o, rs_o = O.quantize_input(x)
     assert_exact(q.cpu().numpy(), q_o, "codes")
     if out == "i32":
-        acc = B.bitlinear_accumulate(q, rs, P_d)
+        acc = B.bitlinear_accumulate(q, rs, P_d, out=guard.empty((M, N), torch.int32))
         assert_exact(acc.cpu().numpy(), O.ternary_matmul(q_o, O.unpack(P_o)), "int32 accumulators")
         return
     y_o = O.forward(x, P_o, beta_o)["y"]
     if out == "f32":
-        y = B.bitlinear_forward_quantized(q, s, rs, P_d, beta, out_dtype=torch.float32)
+        y = B.bitlinear_forward_quantized(q, s, rs, P_d, beta,
+                                          out=guard.empty((M, N), torch.float32))
         assert_f32_output(y.cpu().numpy(), y_o, "gemm f32")
     else:
         r = WL.activations(M, N, seed=M + N) if residual else None
-        y = bf16_dev(r) if residual else torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        y = guard.copy(bf16_dev(r)) if residual else guard.empty((M, N), torch.bfloat16)
         B.bitlinear_forward_quantized(q, s, rs, P_d, beta, residual=y if residual else None, out=y)
         ref = O.residual_add(r, O.f32_to_bf16(y_o)) if residual else O.f32_to_bf16(y_o)
         assert_bf16_output(bf16_host(y), ref, "gemm bf16")

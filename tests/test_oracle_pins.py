@@ -339,6 +339,29 @@ def test_rmsnorm_matches_textbook_formula(O):
     np.testing.assert_allclose(h, ref, rtol=4 * 2.0 ** -24, atol=0)
 
 
+def test_rmsnorm_applies_the_gain_after_the_factor(O):
+    """h = RN32(RN32(x r) g), not RN32(x RN32(r g)): r is recomputed here from
+    the exact sum of squares (math.fsum of exact binary64 squares, then
+    binary64 IEEE divide, add, sqrt, reciprocal, one rounding to binary32), and
+    the row holds elements where the two orders round differently."""
+    import math
+    rng = np.random.default_rng(23)
+    K = 2560
+    xb = bf16(rng.standard_normal((3, K)))
+    gb = bf16(rng.uniform(0.5, 1.5, K))
+    h, r_o = O.rmsnorm(xb, gb, 1e-5)
+    xf, gf = O.bf16_to_f32(xb), O.bf16_to_f32(gb)
+    eps = float(np.float32(1e-5))
+    for m in range(3):
+        ss = math.fsum(float(v) * float(v) for v in xf[m])  # each square exact in binary64
+        r = np.float32(1.0 / math.sqrt(ss / K + eps))
+        assert r == r_o[m]
+        after = ((xf[m] * r).astype(np.float32) * gf).astype(np.float32)
+        before = (xf[m] * np.float32(r * gf.astype(np.float32))).astype(np.float32)
+        assert (after != before).sum() > 10  # the row separates the two orders
+        assert (h[m].view(np.uint32) == after.view(np.uint32)).all()
+
+
 def test_rescale_is_two_correctly_rounded_steps(O):
     """y = RN32(RN32(acc * beta) / s_x), each step the correctly rounded value
     of the exact rational (multiply first, then divide); the other order
@@ -401,6 +424,15 @@ def test_forward_equals_its_steps(O):
 # --------------------------------------------------------------------------
 # FFN block glue
 # --------------------------------------------------------------------------
+# Single-rounding bound of the FFN glue: two binary32 roundings (relative
+# error <= 2^-24 each) and one bf16 rounding (8-bit significand: <= 2^-8) of
+# the exact value give at most 2^-8 + 2^-23 + (smaller terms)
+# < 2^-8 (1 + 2^-14) relative error.  An intermediate rounded to bf16 would
+# double the bf16 term; test_relu2_mul_keeps_the_square_in_binary32 tells the
+# two readings apart bit for bit.
+GLUE_RTOL = 2.0 ** -8 * (1 + 2.0 ** -14)
+
+
 def test_relu2_mul_vs_float64(O):
     rng = np.random.default_rng(41)
     a = bf16(rng.standard_normal(5000) * 3)
@@ -409,8 +441,33 @@ def test_relu2_mul_vs_float64(O):
     af = O.bf16_to_f32(a).astype(np.float64)
     bf = O.bf16_to_f32(b).astype(np.float64)
     ref = np.maximum(af, 0) ** 2 * bf
-    np.testing.assert_allclose(z, ref, rtol=2.0 ** -8, atol=0)
+    np.testing.assert_allclose(z, ref, rtol=GLUE_RTOL, atol=0)
     assert (z[af <= 0] == 0).all()
+
+
+def _torch_bf16_bits(v):
+    """bf16 bits of binary32 values by torch's round-to-nearest-even cast."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(np.asarray(v, np.float32)))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_relu2_mul_keeps_the_square_in_binary32(O):
+    """Pairs where rounding relu(a)^2 to bf16 before the multiply changes the
+    result: the oracle gives the binary32-intermediate value, not the other."""
+    rng = np.random.default_rng(43)
+    a = bf16(np.abs(rng.standard_normal(20000)) * 3 + 0.01)
+    b = bf16(rng.standard_normal(20000) * 3)
+    af, bf = O.bf16_to_f32(a), O.bf16_to_f32(b)
+    sq = (af * af).astype(np.float32)                       # RN32(a^2), a > 0
+    keep = _torch_bf16_bits((sq * bf).astype(np.float32))   # bf16(RN32(RN32(a^2) b))
+    sq_b = O.bf16_to_f32(_torch_bf16_bits(sq))
+    early = _torch_bf16_bits((sq_b * bf).astype(np.float32))  # bf16(RN32(bf16(a^2) b))
+    differ = np.flatnonzero(keep != early)
+    assert differ.size > 100  # the two readings are distinguishable on these inputs
+    z = O.relu2_mul(a[differ], b[differ])
+    assert (z == keep[differ]).all()
+    assert not (z == early[differ]).any()
 
 
 def test_residual_add_vs_float64(O):
@@ -419,7 +476,7 @@ def test_residual_add_vs_float64(O):
     d = bf16(rng.standard_normal(5000) * 0.1)
     out = O.bf16_to_f32(O.residual_add(x, d)).astype(np.float64)
     ref = O.bf16_to_f32(x).astype(np.float64) + O.bf16_to_f32(d).astype(np.float64)
-    np.testing.assert_allclose(out, ref, rtol=2.0 ** -8, atol=0)
+    np.testing.assert_allclose(out, ref, rtol=GLUE_RTOL, atol=0)
 
 
 def _packed(O, W):
