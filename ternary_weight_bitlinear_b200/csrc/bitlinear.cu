@@ -152,13 +152,14 @@ struct WsSlices {
 };
 
 // Tail of a forward workspace used by the 5..64-token kernel when a row tile
-// is shared by several CTAs: one flag and one block of int32 partial sums
-// (npad x 128) per CTA.
+// is shared by several CTAs: one counter and two blocks of int32 partial sums
+// (128 x npad: the tile a CTA's share enters part-way, and the one it leaves
+// part-way) per CTA.
 bool skinny_m(int64_t M) { return M >= kSkMinTokens && M <= kSkMaxTokens; }
 int64_t sk_npad(int64_t M) { return (M + 15) / 16 * 16; }
-int64_t sk_flag_bytes() { return round_up(8 * kSkMaxGrid, 256); }
+int64_t sk_ctr_bytes() { return round_up(8 * kSkMaxGrid, 256); }
 int64_t sk_ws_bytes(int64_t M) {
-    return skinny_m(M) ? sk_flag_bytes() + (int64_t)kSkMaxGrid * sk_npad(M) * 128 * 4 : 0;
+    return skinny_m(M) ? sk_ctr_bytes() + (int64_t)kSkMaxGrid * 2 * 128 * sk_npad(M) * 4 : 0;
 }
 
 WsSlices ws_slices(char* w, int64_t M, int64_t K) {
@@ -396,8 +397,8 @@ bl_status run_gemm(const int8_t* q, const float* s_x, const int32_t* rowsum, con
                   stream, map_q, map_p, map_y, a);
 }
 
-// A launch epoch for the partial-sum flags: never 0 (a cleared flag), and
-// distinct between launches of one process.
+// A launch epoch for the split-tile counters: never 0, and distinct between
+// launches of one process.
 unsigned long long next_epoch() {
     static std::atomic<unsigned long long> e{
         0x9E3779B97F4A7C15ull ^
@@ -451,8 +452,8 @@ bl_status run_skinny(const DecodeJob* jobs, int count, int64_t M, void* ws, size
         b.total = items;
         b.split = split ? 1 : 0;
         if (split) {
-            b.flags = static_cast<unsigned long long*>(ws);
-            b.part = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + sk_flag_bytes());
+            b.ctr = static_cast<unsigned long long*>(ws);
+            b.part = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + sk_ctr_bytes());
         }
         b.epoch = next_epoch();
         const int64_t grid = std::max<int64_t>(

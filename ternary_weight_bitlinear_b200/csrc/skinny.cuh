@@ -8,37 +8,45 @@
 //
 // Design (B200):
 //  * Work unit ("item"): 32 packed rows (= 128 output rows, the MMA's M) x 512
-//    bytes of K of one problem; every item moves the same 16 KB of packed
-//    weights (K past the row end reads as zeros).  Items this large keep the
-//    per-item barrier round trips of the single issuing thread off the
-//    critical path.  The batch's items are laid end to end (problem, row tile, K
-//    stage) and each persistent CTA owns an equal contiguous share, so all SMs
-//    stream the same number of bytes whatever the mix of shapes.
+//    bytes of K of one problem (16 KB of packed weights; the part of the last
+//    item past the row end is neither loaded nor multiplied).  The batch's
+//    items are laid end to end (problem, row tile, K stage) and each
+//    persistent CTA owns an equal contiguous share, so all SMs stream the same
+//    number of bytes whatever the mix of shapes.
+//  * The tensor core costs max(44, N/2) cycles per tcgen05.mma.kind::i8 of
+//    K = 32 on this GPU whatever M (64 or 128) or the source of A (measured).
+//    With the weights as A (M = 128 rows) and the tokens as B (N <= 64), one
+//    instruction takes 1 KB of packed weights per 44 cycles, about the HBM
+//    rate of one SM; the swapped shape (weights as B, N = 256) would take 2 KB
+//    per 128 cycles.  So the weights are A, and the pipeline below exists to
+//    keep that one issuing thread fed.
 //  * Warp 0 loads, per item, the packed tile and the token tile (int8 codes of
-//    all M tokens for those 512 K bytes) with TMA (four 128-byte-swizzled
-//    boxes each, no multicast) into a shared-memory ring, 4 to 8 items deep
-//    depending on M.
+//    all M tokens for those K bytes) with TMA (128-byte swizzled boxes, no
+//    multicast) into a shared-memory ring 4 to 8 items deep.  The packed tiles
+//    of the first ring's worth of items are requested before the kernel waits
+//    on the previous grid (programmatic dependent launch): weights are
+//    constant, so their stream overlaps the quantisation kernel before.
 //  * Two teams of four expansion warps (one per TMEM lane quadrant) alternate
 //    items: each thread reads its packed row, selects its bit pair
-//    (code = t + 1) and writes the 512 codes of its weight row straight into
-//    tensor memory with tcgen05.st -- the expanded weights never touch shared
-//    memory, whose bandwidth is what limits a shared-memory operand here.
-//  * One thread issues tcgen05.mma.cta_group::1.kind::i8 with A (weights,
-//    M=128) from TMEM and B (tokens, N = M rounded up to 16) from shared
-//    memory.  An item's 16 MMAs rotate over 2-4 independent accumulator
-//    chains (double-buffered per row tile) that the epilogue sums.  MMAs this
-//    narrow are bound by their issue rate (~65 cycles each on this GPU,
-//    measured), not by the tensor pipe, which caps this kernel near 0.7 of
-//    the HBM roofline.
-//  * Four epilogue warps take a finished row tile: tcgen05.ld, minus the row
-//    sums, rescale (exact division through the token's reciprocal), store.
-//    A row tile whose items straddle two or more CTAs is finished by the CTA
-//    holding its first items (it reaches them last): the others leave int32
-//    partial sums in the caller's workspace and raise a flag carrying this
-//    launch's epoch; the finisher polls those flags side by side, adds the
-//    sums (16-byte loads of each contributor's block) and clears the flags.
-//    Without a workspace the CTA shares are cut at row-tile boundaries.
-//  * Every wait is bounded (status word + unwind).
+//    (code = t + 1) and writes the codes of its weight row straight into
+//    tensor memory with tcgen05.st (a ring of three 128-column slots), so the
+//    expanded weights never use shared-memory bandwidth.
+//  * One thread issues tcgen05.mma.cta_group::1.kind::i8 with A (weights) from
+//    TMEM and B (tokens, N = M rounded up to 16) from shared memory into one
+//    of two TMEM accumulators, and releases the ring slots with
+//    tcgen05.commit.
+//  * Eight epilogue warps (two per TMEM lane quadrant, each half of the
+//    tokens) take a finished row tile: tcgen05.ld, minus the row sums,
+//    rescale (exact division through the token's reciprocal), store.
+//  * A row tile whose items straddle several CTAs is finished by whichever of
+//    them gets there last: each leaves its int32 partial sums in the caller's
+//    workspace and counts itself in on the tile's counter (an atomic
+//    compare-and-swap that carries this launch's epoch, so no counter needs
+//    clearing); the one that completes the count adds the others' sums and
+//    writes the outputs.  No CTA waits for another, so the kernel needs no
+//    co-residency of its CTAs.  Without a workspace the CTA shares are cut at
+//    row-tile boundaries.
+//  * Every mbarrier wait is bounded (status word + unwind).
 #pragma once
 
 #include <cuda.h>
@@ -58,30 +66,34 @@ constexpr int kSkItemK = kSkKB * kSkBK;              // 512 K bytes per item
 constexpr int kSkMaxStages = 8;                      // shared-memory ring depth (for npad 16)
 constexpr int kSkPBox = kSkRows * kSkBK;             // 4 KB packed box
 constexpr int kSkPBytes = kSkKB * kSkPBox;           // 16 KB packed per item
-constexpr int kSkRingBytes = 196 * 1024;             // ring: (16 KB + 4 * npad * 128) per stage
-constexpr int kSkAStages = 2;                        // TMEM ring of expanded items (128 columns each)
+constexpr int kSkRingBytes = 192 * 1024;             // ring: (16 KB + 4 * npad * 128) per stage
+constexpr int kSkASlots = 3;                         // TMEM ring of expanded items (128 columns each)
 constexpr int kSkTeams = 2;                          // expansion teams (4 warps each)
 constexpr int kSkMmaWarp = 1;
 constexpr int kSkExpWarp0 = 2;
 constexpr int kSkEpiWarp0 = kSkExpWarp0 + 4 * kSkTeams;
-constexpr int kSkThreads = 32 * (kSkEpiWarp0 + 4);
+constexpr int kSkEpiWarps = 8;                       // two per lane quadrant, each half the tokens
+constexpr int kSkEpiThreads = 32 * kSkEpiWarps;
+constexpr int kSkThreads = 32 * (kSkEpiWarp0 + kSkEpiWarps);
 constexpr int kSkCap = 64;                           // problems per launch
 constexpr int kSkMaxGrid = 160;                      // CTAs per launch (>= SM count)
-// TMEM columns: A ring [0, 256); accumulators [256, 512): two buffers of 128
-// columns, each holding 128/stride chains of `stride` = max(32, npad rounded
-// up to 32) columns
+// TMEM columns: A ring [0, 384); accumulators [384, 512): two buffers of 64
 constexpr uint32_t kSkTmemCols = 512;
-constexpr uint32_t kSkDCol0 = 32 * kSkKB * kSkAStages;
-constexpr uint32_t kSkDBuf = 128;
-constexpr int kSkNumBars = 2 * kSkMaxStages + 2 * kSkAStages + 2 * 2 + 1;
+constexpr uint32_t kSkACols = 32 * kSkKB;            // 128 columns (512 K bytes) per slot
+constexpr uint32_t kSkDCol0 = kSkACols * kSkASlots;
+constexpr uint32_t kSkDBuf = 64;
+constexpr int kSkNumBars = 2 * kSkMaxStages + 2 * kSkASlots + 2 * 2 + 1;
 constexpr int kSkOffBar = kSkRingBytes;
-// per-problem token constants for the epilogue: s_x, RN(1/s_x), row sums
-constexpr int kSkOffTok = kSkOffBar + 8 * kSkNumBars + 16;
+// tmem address | last-arriver flag | per-problem token constants (s_x,
+// RN(1/s_x), row sums) for the epilogue
+constexpr int kSkOffTmem = kSkOffBar + 8 * kSkNumBars;
+constexpr int kSkOffTok = kSkOffTmem + 16;
 constexpr int kSkSmemBytes = kSkOffTok + 12 * kSkMaxTokens + 1024;
 static_assert(kSkSmemBytes <= 227 * 1024, "shared memory budget");
 static_assert(kSkPBytes % 1024 == 0, "swizzle atoms stay 1024-aligned");
 static_assert(kSkMaxStages * (kSkPBytes + kSkKB * 16 * kSkBK) <= kSkRingBytes, "ring holds 8 stages at npad 16");
-static_assert(kSkDCol0 + 2 * kSkDBuf <= kSkTmemCols && 2 * kSkMaxTokens <= kSkDBuf, "TMEM budget");
+static_assert(kSkDCol0 + 2 * kSkDBuf <= kSkTmemCols && kSkMaxTokens <= (int)kSkDBuf, "TMEM budget");
+static_assert(kSkThreads * 112 <= 65536, "register budget of one CTA per SM");
 
 struct SkProblem {
     const float* s_x;          // [M]
@@ -108,8 +120,8 @@ struct alignas(64) SkBatch {
     int split;                   // CTA shares may cut row tiles (workspace given)
     int64_t total;               // items in the batch
     unsigned long long epoch;    // nonzero, distinct per launch
-    unsigned long long* flags;   // [gridDim.x] partial-sum flags (split only)
-    int32_t* part;               // [gridDim.x][128][npad] partial sums (split only)
+    unsigned long long* ctr;     // [gridDim.x] split-tile counters (split only)
+    int32_t* part;               // [gridDim.x][2][128][npad] partial sums (split only)
 };
 
 __device__ __forceinline__ int sk_problem_at(const SkBatch& b, int64_t item) {
@@ -131,16 +143,25 @@ __device__ __forceinline__ int64_t sk_share_start(const SkBatch& b, int64_t c, i
     return i;
 }
 
+// The CTA whose share holds `item` (split schedule: shares floor(c T / G)).
+__device__ __forceinline__ int64_t sk_owner(const SkBatch& b, int64_t item, int64_t G) {
+    int64_t c = item * G / b.total;
+    while (c + 1 < G && sk_share_start(b, c + 1, G) <= item) ++c;
+    while (c > 0 && sk_share_start(b, c, G) > item) --c;
+    return c;
+}
+
 // Walk over items: (problem, row tile, K stage).  The current problem's sizes
 // stay in registers: the batch lives in the kernel's parameter block, and
 // indexing it with a runtime problem number on every item costs a
 // constant-cache miss each time.
 struct SkCursor {
-    int p, tile, ks, kst, tiles;
+    int p, tile, ks, kst, tiles, K;
     __device__ __forceinline__ void load(const SkBatch& b) {
         if (p < b.count) {
             kst = b.p[p].kst;
             tiles = b.p[p].tiles;
+            K = b.p[p].K;
         }
     }
     __device__ __forceinline__ void start(const SkBatch& b, int64_t item) {
@@ -160,6 +181,8 @@ struct SkCursor {
             }
         }
     }
+    // K bytes of this item inside the row (1..512)
+    __device__ __forceinline__ int valid_k() const { return min(kSkItemK, K - ks * kSkItemK); }
 };
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -179,6 +202,40 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 16 consecutive 32-bit TMEM columns of this thread's lane (no wait).
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// 8 consecutive 32-bit TMEM columns of this thread's lane (no wait).
+__device__ __forceinline__ void tmem_ld8_nowait(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7])
+                 : "r"(taddr));
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0],"
+        " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+          "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 // A (weights) from TMEM, B (tokens) from shared memory, D in TMEM.
 __device__ __forceinline__ void sk_mma(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -195,34 +252,44 @@ __device__ __forceinline__ uint32_t sk_idesc(int npad) {
     return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(npad >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-// Named barrier among the four epilogue warps, and the same barrier returning
-// whether `pred` held in all of them (so that they always take the same exits
-// and never leave one another waiting at the barrier).
+// Named barrier among the eight epilogue warps.
 __device__ __forceinline__ void sk_epi_sync() {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kSkEpiThreads) : "memory");
 }
 
+// The same barrier, returning whether `pred` held in all of them (so that they
+// always take the same exits and never leave one another waiting).
 __device__ __forceinline__ bool sk_epi_all(bool pred) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred a, b;\n\t"
         "setp.ne.u32 a, %1, 0;\n\t"
-        "bar.red.and.pred b, 1, 128, a;\n\t"
+        "bar.red.and.pred b, 1, %2, a;\n\t"
         "selp.u32 %0, 1, 0, b;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)pred)
+        : "r"((uint32_t)pred), "n"(kSkEpiThreads)
         : "memory");
     return r != 0;
+}
+
+// Count one participant in on a split tile's counter; true for the one that
+// completes the count of n.  The counter's high word holds the launch epoch,
+// so a counter left by an earlier launch (or never written) reads as zero.
+// A compare-and-swap loop: some participant's swap succeeds on every round.
+__device__ __forceinline__ bool sk_arrive_last(unsigned long long* ctr, uint32_t ep, uint32_t n,
+                                               bool& ok) {
+    unsigned long long old = atomicAdd(ctr, 0ull);
+    for (uint32_t it = 0; it < (1u << 20); ++it) {
+        const unsigned long long base =
+            (uint32_t)(old >> 32) == ep ? old : ((unsigned long long)ep << 32);
+        const unsigned long long nv = base + 1ull;
+        const unsigned long long seen = atomicCAS(ctr, old, nv);
+        if (seen == old) return (uint32_t)nv == n;
+        old = seen;
+    }
+    atomicOr(&g_status, kStatusTimeout);
+    ok = false;
+    return false;
 }
 
 // One rescaled output: RN32(RN32(acc * beta) / s_x) through the token's reciprocal.
@@ -264,17 +331,16 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
     auto full_bar = [&](int s) { return bars + 8u * s; };
     auto empty_bar = [&](int s) { return bars + 8u * (kSkMaxStages + s); };
     auto afull_bar = [&](int a) { return bars + 8u * (2 * kSkMaxStages + a); };
-    auto aempty_bar = [&](int a) { return bars + 8u * (2 * kSkMaxStages + kSkAStages + a); };
-    auto dfull_bar = [&](int d) { return bars + 8u * (2 * kSkMaxStages + 2 * kSkAStages + d); };
-    auto dempty_bar = [&](int d) { return bars + 8u * (2 * kSkMaxStages + 2 * kSkAStages + 2 + d); };
-    const uint32_t mma_done_bar = bars + 8u * (2 * kSkMaxStages + 2 * kSkAStages + 4);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSkOffBar + 8 * kSkNumBars);
+    auto aempty_bar = [&](int a) { return bars + 8u * (2 * kSkMaxStages + kSkASlots + a); };
+    auto dfull_bar = [&](int d) { return bars + 8u * (2 * kSkMaxStages + 2 * kSkASlots + d); };
+    auto dempty_bar = [&](int d) { return bars + 8u * (2 * kSkMaxStages + 2 * kSkASlots + 2 + d); };
+    const uint32_t mma_done_bar = bars + 8u * (2 * kSkMaxStages + 2 * kSkASlots + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSkOffTmem);
+    volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(sm + kSkOffTmem + 4);
     // ring stage: 4 packed boxes (4 KB each) | 4 token boxes (npad x 128 each)
     const uint32_t qbox = (uint32_t)(b.npad * kSkBK);
     const uint32_t stage_bytes = (uint32_t)kSkPBytes + kSkKB * qbox;
     const int nstages = min(kSkMaxStages, (int)(kSkRingBytes / stage_bytes));
-    const int dstride = b.npad <= 32 ? 32 : 64;  // accumulator chain width (columns)
-    const int chains = (int)kSkDBuf / dstride;   // 4 or 2
     auto stage_p = [&](int s) { return base + (uint32_t)s * stage_bytes; };
     auto stage_q = [&](int s) { return base + (uint32_t)s * stage_bytes + (uint32_t)kSkPBytes; };
 
@@ -284,13 +350,13 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        for (int a = 0; a < kSkAStages; ++a) {
+        for (int a = 0; a < kSkASlots; ++a) {
             mbar_init(afull_bar(a), 4);
             mbar_init(aempty_bar(a), 1);
         }
         for (int d = 0; d < 2; ++d) {
             mbar_init(dfull_bar(d), 1);
-            mbar_init(dempty_bar(d), 4);
+            mbar_init(dempty_bar(d), kSkEpiWarps);
         }
         mbar_init(mma_done_bar, 1);
         mbar_init_fence();
@@ -301,9 +367,6 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    pdl_wait();
-    pdl_launch_dependents();
-
     const int64_t G = gridDim.x, c = blockIdx.x;
     const int64_t i0 = sk_share_start(b, c, G), i1 = sk_share_start(b, c + 1, G);
     const uint32_t n_items = (uint32_t)(i1 - i0);
@@ -312,17 +375,37 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
+            // the first ring's worth of packed tiles before the wait on the
+            // previous grid (weights are constant), their token tiles after it
+            const uint32_t pre = min(n_items, (uint32_t)nstages);
             SkCursor cur;
             if (n_items) cur.start(b, i0);
-            const uint32_t tx = stage_bytes;  // out-of-range parts of a box are zero-filled, still counted
-            uint32_t g = 0, inflight_from = 0;
+            for (uint32_t g = 0; g < pre; ++g) {
+                const int nkb = (cur.valid_k() + kSkBK - 1) / kSkBK;
+                mbar_arrive_expect_tx(full_bar((int)g), (uint32_t)nkb * ((uint32_t)kSkPBox + qbox));
+                for (int kb = 0; kb < nkb; ++kb)
+                    tma_load_2d(stage_p((int)g) + kb * kSkPBox, &b.tmap_p[cur.p],
+                                cur.ks * kSkItemK + kb * kSkBK, cur.tile * kSkRows, full_bar((int)g));
+                cur.next(b);
+            }
+            pdl_wait();
+            pdl_launch_dependents();
+            if (n_items) cur.start(b, i0);
+            for (uint32_t g = 0; g < pre; ++g) {
+                const int nkb = (cur.valid_k() + kSkBK - 1) / kSkBK;
+                for (int kb = 0; kb < nkb; ++kb)
+                    tma_load_2d(stage_q((int)g) + kb * qbox, &b.tmap_q[cur.p],
+                                cur.ks * kSkItemK + kb * kSkBK, 0, full_bar((int)g));
+                cur.next(b);
+            }
+            uint32_t g = pre, inflight_from = 0;
             for (; g < n_items && ok; ++g) {
                 const int s = (int)(g % (uint32_t)nstages);
                 if (!mbar_wait(empty_bar(s), ((g / nstages) & 1u) ^ 1u)) { ok = false; break; }
-                inflight_from = g >= (uint32_t)nstages ? g - nstages + 1 : 0;
-                mbar_arrive_expect_tx(full_bar(s), tx);
-#pragma unroll
-                for (int kb = 0; kb < kSkKB; ++kb) {
+                inflight_from = g - nstages + 1;
+                const int nkb = (cur.valid_k() + kSkBK - 1) / kSkBK;
+                mbar_arrive_expect_tx(full_bar(s), (uint32_t)nkb * ((uint32_t)kSkPBox + qbox));
+                for (int kb = 0; kb < nkb; ++kb) {
                     const int x = cur.ks * kSkItemK + kb * kSkBK;
                     tma_load_2d(stage_p(s) + kb * kSkPBox, &b.tmap_p[cur.p], x, cur.tile * kSkRows,
                                 full_bar(s));
@@ -330,38 +413,45 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
                 }
                 cur.next(b);
             }
-            if (!ok)
+            if (!ok)  // let the copies still in flight land before the CTA exits
                 for (uint32_t j = inflight_from; j < g; ++j)
                     mbar_wait(full_bar((int)(j % (uint32_t)nstages)), (j / nstages) & 1u);
+        } else {
+            pdl_wait();
+            pdl_launch_dependents();
         }
     } else if (warp == kSkMmaWarp) {
+        pdl_wait();
+        pdl_launch_dependents();
         // ---------------- MMA issuer ----------------
+        // Kept small on purpose: ring positions and phases are counters, and
+        // the MMAs of an item are one rolled loop, so that this thread's code
+        // stays in the instruction cache next to the other roles' code.
         if (lane == 0) {
             SkCursor cur;
             if (n_items) cur.start(b, i0);
             const uint32_t idesc = sk_idesc(b.npad);
-            uint32_t tl = 0;
+            const uint32_t qstep = qbox >> 4;  // descriptor address units between token boxes
+            int s = 0, a = 0, d = 0;
+            uint32_t sph = 0, aph = 0, dph = 0;
             bool first = true;
             for (uint32_t g = 0; g < n_items && ok; ++g) {
-                const int s = (int)(g % (uint32_t)nstages), a = (int)(g % kSkAStages), d = (int)(tl & 1);
-                if (first && !mbar_wait(dempty_bar(d), ((tl >> 1) & 1u) ^ 1u)) { ok = false; break; }
-                if (!mbar_wait(full_bar(s), (g / nstages) & 1u) ||
-                    !mbar_wait(afull_bar(a), (g / kSkAStages) & 1u)) {
+                if (first && !mbar_wait(dempty_bar(d), dph ^ 1u)) { ok = false; break; }
+                if (!mbar_wait(afull_bar(a), aph) || !mbar_wait(full_bar(s), sph)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t dcol = tmem + kSkDCol0 + (uint32_t)d * kSkDBuf;
-#pragma unroll
-                for (int kb = 0; kb < kSkKB; ++kb) {
-                    const uint64_t bd = smem_desc_sw128(stage_q(s) + kb * qbox);
-#pragma unroll
-                    for (int kk = 0; kk < kSkBK / 32; ++kk) {  // 32 K bytes = 8 TMEM columns of A
-                        const int t = kb * (kSkBK / 32) + kk;  // MMA number in the item
-                        const int ch = t & (chains - 1);
-                        sk_mma(dcol + (uint32_t)(ch * dstride), tmem + (uint32_t)(32 * kSkKB * a + 8 * t),
-                               bd + 2u * kk, idesc, (first && t < chains) ? 0u : 1u);
-                    }
+                uint32_t acol = tmem + kSkACols * (uint32_t)a;  // 32 K bytes = 8 TMEM columns of A
+                const uint64_t bd = smem_desc_sw128(stage_q(s));
+                const int nmma = (cur.valid_k() + 31) >> 5;
+                uint32_t acc = first ? 0u : 1u;
+#pragma unroll 1
+                for (int t = 0; t < nmma; ++t) {
+                    sk_mma(dcol, acol, bd + 2u * (uint32_t)(t & 3) + qstep * (uint32_t)(t >> 2), idesc, acc);
+                    acc = 1u;
+                    acol += 8u;
                 }
                 tc_commit(empty_bar(s));
                 tc_commit(aempty_bar(a));
@@ -369,27 +459,36 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
                 first = last;
                 if (last) {
                     tc_commit(dfull_bar(d));
-                    ++tl;
+                    if ((d ^= 1) == 0) dph ^= 1u;
                 }
+                if (++s == nstages) { s = 0; sph ^= 1u; }
+                if (++a == kSkASlots) { a = 0; aph ^= 1u; }
                 cur.next(b);
             }
             tc_commit(mma_done_bar);
             mbar_wait(mma_done_bar, 0);
         }
     } else if (warp < kSkEpiWarp0) {
+        pdl_wait();
+        pdl_launch_dependents();
         // ---------------- expansion teams ----------------
         const int team = (warp - kSkExpWarp0) >> 2, qd = warp & 3;
         const int bit = lane >> 3, j = lane & 7;  // this lane: bit pair, packed row 8*qd + j
         const int prow = 8 * qd + j;
         const uint32_t tlane = (uint32_t)(32 * qd) << 16;
+        SkCursor cur;
+        if (n_items > (uint32_t)team) {
+            cur.start(b, i0);
+            if (team) cur.next(b);
+        }
         for (uint32_t g = (uint32_t)team; g < n_items && ok; g += kSkTeams) {
-            const int s = (int)(g % (uint32_t)nstages), a = (int)(g % kSkAStages);
+            const int s = (int)(g % (uint32_t)nstages), a = (int)(g % kSkASlots);
             const bool got = mbar_wait(full_bar(s), (g / nstages) & 1u) &&
-                             mbar_wait(aempty_bar(a), ((g / kSkAStages) & 1u) ^ 1u);
+                             mbar_wait(aempty_bar(a), ((g / kSkASlots) & 1u) ^ 1u);
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
-#pragma unroll
-            for (int kb = 0; kb < kSkKB; ++kb) {
+            const int nkb = (cur.valid_k() + kSkBK - 1) / kSkBK;
+            for (int kb = 0; kb < nkb; ++kb) {
                 const uint8_t* pk = sm + (size_t)s * stage_bytes + kb * kSkPBox + prow * kSkBK;
                 uint32_t w[32];
 #pragma unroll
@@ -400,22 +499,31 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
                     w[4 * ch + 2] = (v.z >> (2 * bit)) & 0x03030303u;
                     w[4 * ch + 3] = (v.w >> (2 * bit)) & 0x03030303u;
                 }
-                tmem_st32(tmem + tlane + (uint32_t)(32 * kSkKB * a + 32 * kb), w);
+                tmem_st32(tmem + tlane + kSkACols * (uint32_t)a + 32u * (uint32_t)kb, w);
             }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(afull_bar(a));
+            cur.next(b);
+            cur.next(b);
         }
     } else {
-        // ---------------- epilogue: one weight row per thread ----------------
-        const int qd = warp & 3;
+        pdl_wait();
+        pdl_launch_dependents();
+        // ---------------- epilogue: one weight row, half of the tokens per thread ----------------
+        const int ew = warp - kSkEpiWarp0;
+        const int qd = warp & 3, half = ew >> 2;
         const int bit = lane >> 3, j = lane & 7;
         const int row128 = 32 * qd + lane;  // D row (TMEM lane)
         float* tok_s = reinterpret_cast<float*>(sm + kSkOffTok);
         float* tok_y = tok_s + kSkMaxTokens;
         int* tok_rs = reinterpret_cast<int*>(tok_y + kSkMaxTokens);
-        const int et = threadIdx.x - 32 * kSkEpiWarp0;  // 0..127
+        const int et = threadIdx.x - 32 * kSkEpiWarp0;  // 0..255
+        // this thread's token columns [c0, c1): halves of npad in 16-column steps
+        const int hc = ((b.npad / 2) + 15) & ~15;
+        const int c0 = half * hc, c1 = min(b.npad, c0 + hc);
+        const uint32_t ep32 = (uint32_t)b.epoch;
         int staged = -1;
         SkCursor cur;
         if (n_items) cur.start(b, i0);
@@ -439,93 +547,86 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
             const int64_t tile_first = pr.item0 + (int64_t)cur.tile * pr.kst;
             const int64_t tile_end = tile_first + pr.kst;
             const int64_t part_end = min(tile_end, i1);
-            const bool started_before = item > tile_first;
-            const bool continues = part_end < tile_end;
+            const bool split = item > tile_first || part_end < tile_end;
             const int d = (int)(tl & 1);
             const bool got = mbar_wait(dfull_bar(d), (tl >> 1) & 1u);
             if (!sk_epi_all(got)) { ok = false; break; }
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(32 * qd) << 16) + kSkDCol0 + (uint32_t)d * kSkDBuf;
-            // a finisher first waits for the partial sums of every later CTA
-            // whose share starts inside this tile (CTAs c+1 .. c_end-1); the
-            // lanes of the first epilogue warp poll those flags side by side
-            int64_t c_end = c + 1;
-            bool waited = true;
-            if (!started_before && continues) {
-                while (c_end < G && sk_share_start(b, c_end, G) < tile_end) ++c_end;
-                if (warp == kSkEpiWarp0) {
-                    const unsigned long long t0 = globaltimer_ns();
-                    for (int64_t c2 = c + 1 + lane; c2 < c_end && waited; c2 += 32) {
-                        while (ld_acquire_u64(b.flags + c2) != b.epoch) {
-                            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                                atomicOr(&g_status, kStatusTimeout);
-                                waited = false;
-                                break;
+            bool write = true;
+            if (split) {
+                // leave this CTA's partial sums, count in; the last one to
+                // arrive adds the others' sums into its accumulator and writes
+                const int64_t cf = sk_owner(b, tile_first, G), cl = sk_owner(b, tile_end - 1, G);
+                const int role = item > tile_first ? 0 : 1;
+                uint32_t v[32];
+                if (c0 < c1) {
+                    tmem_ld16_nowait(taddr + (uint32_t)c0, v);
+                    if (c1 - c0 > 16) tmem_ld16_nowait(taddr + (uint32_t)(c0 + 16), v + 16);
+                    tmem_ld_wait();
+                }
+                int32_t* mine = b.part + ((size_t)(2 * c + role) * 128 + row128) * b.npad;
+#pragma unroll
+                for (int k = 0; k < 32; k += 4)
+                    if (c0 + k < c1)
+                        *reinterpret_cast<uint4*>(mine + c0 + k) = make_uint4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+                __threadfence();
+                sk_epi_sync();
+                if (et == 0) {
+                    bool aok = true;
+                    *last_flag = sk_arrive_last(b.ctr + cf, ep32, (uint32_t)(cl - cf + 1), aok) ? 1u : 0u;
+                    if (!aok) *last_flag = 2u;
+                }
+                sk_epi_sync();
+                const uint32_t lf = *last_flag;
+                if (lf == 2u) ok = false;
+                write = lf == 1u;
+                if (write) {
+                    __threadfence();
+                    for (int64_t c2 = cf; c2 <= cl; ++c2) {
+                        if (c2 == c) continue;
+                        const int32_t* other =
+                            b.part + ((size_t)(2 * c2 + (c2 == cf ? 1 : 0)) * 128 + row128) * b.npad;
+#pragma unroll
+                        for (int k = 0; k < 32; k += 4) {
+                            if (c0 + k < c1) {
+                                const uint4 w4 = __ldcg(reinterpret_cast<const uint4*>(other + c0 + k));
+                                v[k] += w4.x;
+                                v[k + 1] += w4.y;
+                                v[k + 2] += w4.z;
+                                v[k + 3] += w4.w;
                             }
                         }
                     }
+                    // the tile's sums back into the accumulator, read below like any other
+                    if (c0 < c1) {
+                        tmem_st16(taddr + (uint32_t)c0, v);
+                        if (c1 - c0 > 16) tmem_st16(taddr + (uint32_t)(c0 + 16), v + 16);
+                        tmem_st_wait();
+                    }
                 }
-                waited = sk_epi_all(waited);  // also orders the flags before the reads
             }
             const int r = cur.tile * kSkRows + 8 * qd + j;  // packed row
-            const int64_t n = (int64_t)bit * pr.R + r;
-            const int halves = (b.npad + 31) >> 5;
-            for (int h = 0; h < halves; ++h) {  // 32 tokens at a time
-                uint32_t v[32];
-                tmem_ld32(taddr + (uint32_t)(32 * h), v);
-                for (int ch = 1; ch < chains; ++ch) {  // sum the accumulator chains
-                    uint32_t u[32];
-                    tmem_ld32(taddr + (uint32_t)(ch * dstride + 32 * h), u);
-#pragma unroll
-                    for (int m = 0; m < 32; ++m) v[m] += u[m];
-                }
-                if (started_before) {
-                    // contributor: leave the partial sums for the tile's finisher,
-                    // each weight row's npad sums contiguous (16-byte stores)
-                    uint4* dst = reinterpret_cast<uint4*>(b.part + ((size_t)c * 128 + row128) * b.npad + 32 * h);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        if (32 * h + 4 * k < b.npad)
-                            dst[k] = make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-                } else if (waited) {
-                    // one contributor at a time, all of its 16-byte loads in flight
-                    for (int64_t c2 = c + 1; c2 < c_end; ++c2) {
-                        const uint4* src =
-                            reinterpret_cast<const uint4*>(b.part + ((size_t)c2 * 128 + row128) * b.npad + 32 * h);
-                        uint4 w[8];
-#pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            w[k] = 32 * h + 4 * k < b.npad ? __ldcg(src + k) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            v[4 * k] += w[k].x;
-                            v[4 * k + 1] += w[k].y;
-                            v[4 * k + 2] += w[k].z;
-                            v[4 * k + 3] += w[k].w;
-                        }
-                    }
+            if (write) {  // warp-uniform: the TMEM loads are warp-wide, the stores per lane
+                // eight tokens at a time from TMEM, in a rolled loop (small code)
+                const int64_t n = (int64_t)bit * pr.R + r;
+                const int cend = min(c1, b.M);
+#pragma unroll 1
+                for (int cg = c0; cg < cend; cg += 8) {
+                    uint32_t v8[8];
+                    tmem_ld8_nowait(taddr + (uint32_t)cg, v8);
+                    tmem_ld_wait();
                     if (r < pr.R) {
 #pragma unroll
-                        for (int m = 0; m < 32; ++m) {
-                            const int mm = 32 * h + m;
-                            if (mm < b.M) sk_store(pr, mm, n, (int)v[m] - tok_rs[mm], tok_s[mm], tok_y[mm]);
-                        }
+                        for (int k = 0; k < 8; ++k)
+                            if (cg + k < cend)
+                                sk_store(pr, cg + k, n, (int)v8[k] - tok_rs[cg + k], tok_s[cg + k], tok_y[cg + k]);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(dempty_bar(d));
-            if (started_before) {  // raise this CTA's flag once all four warps wrote
-                __threadfence();
-                sk_epi_sync();
-                if (warp == kSkEpiWarp0 && lane == 0) st_release_u64(b.flags + c, b.epoch);
-            } else if (continues) {
-                sk_epi_sync();  // every warp has read before the flags are cleared
-                if (threadIdx.x == kSkEpiWarp0 * 32)
-                    for (int64_t c2 = c + 1; c2 < c_end; ++c2) b.flags[c2] = 0ull;
-                if (!waited) ok = false;
-            }
+            if (lane == 0) mbar_arrive(dempty_bar(d));  // the accumulator is free again
             // next part
             for (int64_t k = item; k < part_end; ++k) cur.next(b);
             item = part_end;
