@@ -224,6 +224,49 @@ bl_status bitlinear_forward_quantized(const int8_t* q, const float* s_x, const i
 bl_status bitlinear_accumulate(const int8_t* q, const int32_t* rowsum, const uint8_t* P,
                                int64_t M, int64_t K, int64_t N, int32_t* acc, void* stream);
 
+/* ---- the FFN block's gate/up pair in one pass ---------------------------- */
+
+/* Workspace bitlinear_pack_gate_up needs for two [I,K] master weights. */
+bl_status bitlinear_pack_gate_up_workspace_size(int64_t I, int64_t K, size_t* bytes);
+
+/* The gate and up projections of an FFN block ([MD] model details: gated
+ * ReLU^2 FFN) packed as one matrix: each ternarised with its own absmean
+ * scale exactly as bitlinear_pack does, then packed as the concatenation
+ * [gate; up] ([2I, K], the layout of bitlinear_pack).  With the block layout
+ * ([BG] pack_weights, "推理侧 BitLinear") bit pairs 0 and 1 of packed row r
+ * hold gate rows r and I/2 + r and bit pairs 2 and 3 the up rows with the
+ * same indices, so one byte carries both operands of two outputs of
+ * relu(gate)^2 * up.
+ *   W_gate, W_up  device fp32 [I,K] master weights; I even.
+ *   P2            device uint8 [I/2, K] output (bitlinear_pack_ternary of the
+ *                 concatenated ternary matrices gives the same bytes).
+ *   beta_out      device float[2] output: {beta_gate, beta_up}.
+ *   workspace     device, >= bitlinear_pack_gate_up_workspace_size bytes. */
+bl_status bitlinear_pack_gate_up(const float* W_gate, const float* W_up, int64_t I, int64_t K,
+                                 uint8_t* P2, float* beta_out, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* The gate and up BitLinear projections of one quantised input and the gated
+ * squared ReLU of the FFN block, in one pass over the pair's packed weights
+ * ([BG] "推理侧 BitLinear" for each projection, [MD] model details for the
+ * relu^2 gating):
+ *   g = bf16(RN32(RN32(acc_gate * beta_gate) / s_x)),
+ *   u = bf16(RN32(RN32(acc_up * beta_up) / s_x)),
+ *   z[m, n] = bf16(RN32(RN32(relu(g) * relu(g)) * u)),  n < I,
+ * bit for bit what bitlinear_forward_quantized of each projection followed by
+ * bitlinear_relu2_mul gives, without writing g and u to memory.
+ *   q, s_x, rowsum  as for bitlinear_forward_quantized (device).
+ *   P2              device uint8 [I/2, K] from bitlinear_pack_gate_up.
+ *   z               device bf16 [M, I] output.
+ *   workspace       device or NULL: for 5 <= M <= 64, at least
+ *                   bitlinear_quantized_batch_workspace_size(M) bytes give
+ *                   every CTA an equal share of the weights (as for the
+ *                   quantized batch); NULL cuts shares at row tiles. */
+bl_status bitlinear_forward_gate_up(const int8_t* q, const float* s_x, const int32_t* rowsum,
+                                    const uint8_t* P2, float beta_gate, float beta_up, int64_t M,
+                                    int64_t K, int64_t I, uint16_t* z, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
 /* ---- forward without any caller-provided memory besides inputs and outputs -- */
 
 /* Size of the library's fixed device scratch used by bitlinear_forward_noalloc. */

@@ -7,7 +7,9 @@ from .bitlinear import (BL_MAX_K, BL_OUT_BF16, BL_OUT_F32, BitLinearError, LIB_P
                         bitlinear_accumulate, bitlinear_act_quant, bitlinear_device_status,
                         bitlinear_forward, bitlinear_forward_batch,
                         bitlinear_forward_batch_workspace_size, bitlinear_forward_quantized,
-                        bitlinear_forward_quantized_batch, make_batch,
+                        bitlinear_forward_quantized_batch, bitlinear_forward_gate_up,
+                        bitlinear_pack_gate_up, bitlinear_pack_gate_up_workspace_size,
+                        make_batch,
                         make_quantized_batch,
                         bitlinear_forward_workspace_size, bitlinear_pack,
                         bitlinear_pack_ternary, bitlinear_pack_workspace_size,

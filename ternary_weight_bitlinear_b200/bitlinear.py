@@ -38,6 +38,10 @@ SIGNATURES = {
                                     _INT),
     "bitlinear_accumulate": ([_P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "bitlinear_relu2_mul": ([_P, _P, _I64, _P, _P], _INT),
+    "bitlinear_pack_gate_up_workspace_size": ([_I64, _I64, ctypes.POINTER(_SZ)], _INT),
+    "bitlinear_pack_gate_up": ([_P, _P, _I64, _I64, _P, _P, _P, _SZ, _P], _INT),
+    "bitlinear_forward_gate_up": ([_P, _P, _P, _P, _F32, _F32, _I64, _I64, _I64, _P, _P, _SZ, _P],
+                                  _INT),
     "bitlinear_forward_noalloc": ([_P, _P, _F32, _P, _F32, _I64, _I64, _I64, _P, _INT, _P], _INT),
     "bitlinear_device_status": ([_P], _INT),
     "bitlinear_selftest_wait_timeout": ([_I64, _P], _INT),
@@ -301,6 +305,43 @@ def bitlinear_relu2_mul(a, b, out=None, stream=None):
     z = torch.empty_like(a) if out is None else out
     _check("bitlinear_relu2_mul", lib().bitlinear_relu2_mul(_ptr(a), _ptr(b), a.numel(), _ptr(z),
                                                             _stream(stream)))
+    return z
+
+
+def bitlinear_pack_gate_up_workspace_size(I, K):
+    n = ctypes.c_size_t()
+    _check("bitlinear_pack_gate_up_workspace_size",
+           lib().bitlinear_pack_gate_up_workspace_size(I, K, ctypes.byref(n)))
+    return n.value
+
+
+def bitlinear_pack_gate_up(W_gate, W_up, P2=None, beta=None, workspace=None, stream=None):
+    """fp32 masters W_gate, W_up [I,K] -> (P2 uint8 [I/2,K], beta fp32 [2] = {gate, up})."""
+    _need(W_gate, torch.float32, "W_gate", 2)
+    _need(W_up, torch.float32, "W_up", 2)
+    I, K = W_gate.shape
+    if W_up.shape != W_gate.shape:
+        raise TypeError("W_gate and W_up must have the same shape")
+    P2 = torch.empty((I // 2, K), dtype=torch.uint8, device=W_gate.device) if P2 is None else P2
+    beta = torch.empty(2, dtype=torch.float32, device=W_gate.device) if beta is None else beta
+    ws = _workspace(bitlinear_pack_gate_up_workspace_size(I, K), W_gate.device) \
+        if workspace is None else workspace
+    _check("bitlinear_pack_gate_up", lib().bitlinear_pack_gate_up(
+        _ptr(W_gate), _ptr(W_up), I, K, _ptr(P2), _ptr(beta), _ptr(ws), ws.numel(), _stream(stream)))
+    return P2, beta
+
+
+def bitlinear_forward_gate_up(q, s_x, rowsum, P2, beta_gate, beta_up, out=None, workspace=None,
+                              stream=None):
+    """z = relu(gate)^2 * up (bf16 [M, I]) from quantised activations and a packed pair."""
+    _need(q, torch.int8, "q", 2)
+    _need(P2, torch.uint8, "P2", 2)
+    M, K = q.shape
+    I = 2 * P2.shape[0]
+    z = torch.empty((M, I), dtype=torch.bfloat16, device=q.device) if out is None else out
+    _check("bitlinear_forward_gate_up", lib().bitlinear_forward_gate_up(
+        _ptr(q), _ptr(s_x), _ptr(rowsum), _ptr(P2), float(beta_gate), float(beta_up), M, K, I,
+        _ptr(z), _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream)))
     return z
 
 

@@ -230,9 +230,12 @@ struct DecodeJob {
     const uint8_t* P;
     void* y;
     const uint16_t* residual;
-    int64_t K, N;
+    int64_t K, N;   // N outputs per token
     float beta;
     int epi;
+    float beta2 = 0.0f;  // kEpiGateUp: the up projection's scale
+    // packed rows of P: N/4, or N/2 for a gate/up pair (N = the pair's I outputs)
+    int64_t packed_rows() const { return epi == kEpiGateUp ? N / 2 : N / 4; }
 };
 
 template <int MT, int CAP>
@@ -261,11 +264,12 @@ bl_status launch_decode_cap(const DecodeJob* jobs, int count, int mt, int dev,
         p.P = jobs[i].P;
         p.y = jobs[i].y;
         p.residual = jobs[i].residual;
-        p.R = jobs[i].N / 4;
+        p.R = jobs[i].packed_rows();
         p.N = jobs[i].N;
         p.byte0 = total;
         p.K = (int)jobs[i].K;
         p.beta = jobs[i].beta;
+        p.beta2 = jobs[i].beta2;
         p.epi = jobs[i].epi;
         total += p.R * p.K;
         rows += p.R;
@@ -346,39 +350,44 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType type, uint64_t elem_bytes
     return true;
 }
 
-bl_status run_gemm(const int8_t* q, const float* s_x, const int32_t* rowsum, const uint8_t* P,
-                   float beta, int64_t M, int64_t K, int64_t N, void* y, int epi,
-                   const uint16_t* residual, int dev, const DeviceInfo& info,
+bl_status run_gemm(const DecodeJob& j, int64_t M, int dev, const DeviceInfo& info,
                    cudaStream_t stream) {
+    const int8_t* q = j.q;
+    const uint8_t* P = j.P;
+    void* y = j.y;
+    const uint16_t* residual = j.residual;
+    const int64_t K = j.K, N = j.N, R = j.packed_rows();
+    const int epi = j.epi;
     CUtensorMap map_q, map_p;
     if (!make_map_u8(&map_q, q, (uint64_t)K, (uint64_t)M, kTcBK, kTcBM,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_u8(&map_p, P, (uint64_t)K, (uint64_t)(N / 4), kTcBK, kTcPackRows,
+        !make_map_u8(&map_p, P, (uint64_t)K, (uint64_t)R, kTcBK, kTcPackRows,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
         return BL_ERR_CUDA;
     TcArgs a = {};
     a.P = P;
-    a.s_x = s_x;
-    a.rowsum = rowsum;
+    a.s_x = j.s_x;
+    a.rowsum = j.rowsum;
     a.y = y;
     a.residual = residual;
-    a.beta = beta;
+    a.beta = j.beta;
+    a.beta2 = j.beta2;
     a.epi = epi;
     a.M = (int)M;
     a.K = (int)K;
-    a.R = (int)(N / 4);
+    a.R = (int)R;
     a.N = N;
-    a.tiles_n = (int)((N / 4 + kTcPackRows - 1) / kTcPackRows);
+    a.tiles_n = (int)((R + kTcPackRows - 1) / kTcPackRows);
     a.tiles_m = (int)((M + kTcBM - 1) / kTcBM);
     // 16-byte output accesses need every run of 32 outputs to start 16-byte aligned
-    const int64_t out_bytes = epi == kEpiBF16 ? 2 : 4;
-    a.vec_ok = ((N / 4) * out_bytes % 16 == 0) && (N * out_bytes % 16 == 0) &&
+    const int64_t out_bytes = (epi == kEpiBF16 || epi == kEpiGateUp) ? 2 : 4;
+    a.vec_ok = (R * out_bytes % 16 == 0) && (N * out_bytes % 16 == 0) &&
                (reinterpret_cast<uintptr_t>(y) % 16 == 0) &&
                (!residual || reinterpret_cast<uintptr_t>(residual) % 16 == 0);
     // bf16 y without a residual leaves through TMA stores of 32 x 32 chunks
     // (column offsets i*R + r are multiples of 8 elements when vec_ok holds)
     CUtensorMap map_y = map_q;
-    if (a.vec_ok && epi == kEpiBF16 && !residual) {
+    if (a.vec_ok && (epi == kEpiBF16 || epi == kEpiGateUp) && !residual) {
         if (!make_map_2d(&map_y, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, y, (uint64_t)N, (uint64_t)M, 32,
                          32, CU_TENSOR_MAP_SWIZZLE_64B))
             return BL_ERR_CUDA;
@@ -435,11 +444,12 @@ bl_status run_skinny(const DecodeJob* jobs, int count, int64_t M, void* ws, size
             p.y = j.y;
             p.residual = j.residual;
             p.N = j.N;
-            p.R = (int)(j.N / 4);
+            p.R = (int)j.packed_rows();
             p.K = (int)j.K;
             p.tiles = (p.R + kSkRows - 1) / kSkRows;
             p.kst = (p.K + kSkItemK - 1) / kSkItemK;
             p.beta = j.beta;
+            p.beta2 = j.beta2;
             p.epi = j.epi;
             p.item0 = items;
             items += (int64_t)p.tiles * p.kst;
@@ -469,15 +479,19 @@ bl_status run_skinny(const DecodeJob* jobs, int count, int64_t M, void* ws, size
 // for up to four tokens, the weight-streaming tensor-core kernel for 5..64,
 // the tensor-core GEMM beyond.  sk_ws: the optional split workspace of the
 // 5..64-token kernel.
+bl_status run_job(const DecodeJob& j, int64_t M, int dev, const DeviceInfo& info,
+                  cudaStream_t stream, void* sk_ws = nullptr, size_t sk_ws_len = 0) {
+    if (M > kSkMaxTokens) return run_gemm(j, M, dev, info, stream);
+    if (M > kDecMaxTokens) return run_skinny(&j, 1, M, sk_ws, sk_ws_len, dev, info, stream);
+    return run_decode(&j, 1, (int)M, dev, info, stream);
+}
+
 bl_status run_quantized(const int8_t* q, const float* s_x, const int32_t* rowsum, const uint8_t* P,
                         float beta, int64_t M, int64_t K, int64_t N, void* y, int epi,
                         const uint16_t* residual, int dev, const DeviceInfo& info,
                         cudaStream_t stream, void* sk_ws = nullptr, size_t sk_ws_len = 0) {
-    DecodeJob j = {q, s_x, rowsum, P, y, residual, K, N, beta, epi};
-    if (M > kSkMaxTokens)
-        return run_gemm(q, s_x, rowsum, P, beta, M, K, N, y, epi, residual, dev, info, stream);
-    if (M > kDecMaxTokens) return run_skinny(&j, 1, M, sk_ws, sk_ws_len, dev, info, stream);
-    return run_decode(&j, 1, (int)M, dev, info, stream);
+    const DecodeJob j = {q, s_x, rowsum, P, y, residual, K, N, beta, epi};
+    return run_job(j, M, dev, info, stream, sk_ws, sk_ws_len);
 }
 
 int epi_of(bl_out_dtype d) {
@@ -560,8 +574,57 @@ bl_status bitlinear_pack(const float* W, int64_t N, int64_t K, uint8_t* P, float
                      beta_out)) != BL_OK)
         return st;
     const int64_t R = N / 4, work = R * (K / 16);
+    PackSlots sl;
+    for (int i = 0; i < 4; ++i) {
+        sl.src[i] = W + (int64_t)i * R * K;
+        sl.ws[i] = ws;
+    }
     return launch(ternarize_pack_kernel, dim3((unsigned)((work + kPackThreads - 1) / kPackThreads)),
-                  dim3(kPackThreads), 0, s, W, R, K, (const PackWorkspace*)ws, P);
+                  dim3(kPackThreads), 0, s, sl, R, K, P);
+}
+
+bl_status bitlinear_pack_gate_up_workspace_size(int64_t I, int64_t K, size_t* bytes) {
+    if (!bytes) return BL_ERR_NULL;
+    bl_status st = check_shape(0, K, 2 * I);
+    if (st != BL_OK) return st;
+    if (I % 2 != 0) return BL_ERR_SHAPE;
+    *bytes = 2 * sizeof(PackWorkspace);
+    return BL_OK;
+}
+
+bl_status bitlinear_pack_gate_up(const float* W_gate, const float* W_up, int64_t I, int64_t K,
+                                 uint8_t* P2, float* beta_out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    size_t need = 0;
+    bl_status st = bitlinear_pack_gate_up_workspace_size(I, K, &need);
+    if (st != BL_OK) return st;
+    if (!W_gate || !W_up || !P2 || !beta_out) return BL_ERR_NULL;
+    if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(W_gate) || !aligned16(W_up) || !aligned16(P2) || !aligned16(workspace))
+        return BL_ERR_ALIGN;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    PackWorkspace* ws = static_cast<PackWorkspace*>(workspace);
+    const float* W[2] = {W_gate, W_up};
+    const int64_t n = I * K;
+    for (int h = 0; h < 2; ++h) {  // each projection's own absmean scale
+        if ((st = launch(absmean_partial_kernel, dim3(kPackPartials), dim3(kPackThreads), 0, s, W[h],
+                         n, ws + h)) != BL_OK)
+            return st;
+        if ((st = launch(absmean_finalize_kernel, dim3(1), dim3(32), 0, s, n, kPackPartials, ws + h,
+                         beta_out + h)) != BL_OK)
+            return st;
+    }
+    const int64_t R = I / 2, work = R * (K / 16);  // packed rows of the [2I, K] concatenation
+    PackSlots sl;
+    for (int i = 0; i < 4; ++i) {
+        sl.src[i] = W[i >> 1] + (int64_t)(i & 1) * R * K;
+        sl.ws[i] = ws + (i >> 1);
+    }
+    return launch(ternarize_pack_kernel, dim3((unsigned)((work + kPackThreads - 1) / kPackThreads)),
+                  dim3(kPackThreads), 0, s, sl, R, K, P2);
 }
 
 bl_status bitlinear_pack_ternary(const int8_t* t, int64_t N, int64_t K, uint8_t* P, void* stream) {
@@ -738,6 +801,26 @@ bl_status bitlinear_forward_quantized(const int8_t* q, const float* s_x, const i
     if ((st = current_device(&dev, &info)) != BL_OK) return st;
     return run_quantized(q, s_x, rowsum, P, beta, M, K, N, y, epi, residual, dev, info,
                          static_cast<cudaStream_t>(stream));
+}
+
+bl_status bitlinear_forward_gate_up(const int8_t* q, const float* s_x, const int32_t* rowsum,
+                                    const uint8_t* P2, float beta_gate, float beta_up, int64_t M,
+                                    int64_t K, int64_t I, uint16_t* z, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+    bl_status st = check_shape(M, K, 2 * I);
+    if (st != BL_OK) return st;
+    if (I % 2 != 0) return BL_ERR_SHAPE;
+    if (M == 0) return BL_OK;
+    if (!q || !s_x || !rowsum || !P2 || !z) return BL_ERR_NULL;
+    if (!aligned16(q) || !aligned16(P2) || !aligned16(z) || (workspace && !aligned16(workspace)))
+        return BL_ERR_ALIGN;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    DecodeJob j = {q, s_x, rowsum, P2, z, nullptr, K, I, beta_gate, kEpiGateUp};
+    j.beta2 = beta_up;
+    return run_job(j, M, dev, info, static_cast<cudaStream_t>(stream), workspace,
+                   workspace ? workspace_bytes : 0);
 }
 
 bl_status bitlinear_quantized_batch_workspace_size(int64_t M, size_t* bytes) {

@@ -209,6 +209,15 @@ __device__ __noinline__ float scale_slow(int acc, float beta, float s, float y) 
     return recip_div(__fmul_rn(__int2float_rn(acc), beta), RecipDiv{s, y});
 }
 
+// The gated squared-ReLU of the FFN block ("BitNet" transformers model doc,
+// model details: hidden_act relu2, gated): z = bf16(RN32(RN32(relu(a)^2) * b))
+// for bf16 a (gate output) and b (up output).
+__device__ __forceinline__ uint16_t relu2_mul_one(uint32_t a_bits, uint32_t b_bits) {
+    const float av = bf16_bits_to_float(a_bits);
+    const float ra = av > 0.0f ? av : 0.0f;
+    return float_to_bf16_bits(__fmul_rn(__fmul_rn(ra, ra), bf16_bits_to_float(b_bits)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -71,7 +71,11 @@ static_assert(8 * kDecWarps * kDecSlots <= kDecBarBytes, "barriers overlap the s
 static_assert(kDecBarBytes % 128 == 0 && kDecChunk % 16 == 0, "copy alignment");
 static_assert(kDecSmemBytes <= 227 * 1024, "shared memory budget");
 
-enum Epilogue { kEpiF32 = 0, kEpiBF16 = 1, kEpiI32 = 2 };
+// Output kinds.  kEpiGateUp: the packed matrix is a gate/up pair packed as
+// [gate; up] (bit pairs 0, 1 gate rows r and R + r, bit pairs 2, 3 the up rows),
+// and the output is z[m, i*R + r] = relu2_mul(bf16 gate, bf16 up) for i = 0, 1
+// (N = 2R outputs), the up rows rescaled with their own scale beta2.
+enum Epilogue { kEpiF32 = 0, kEpiBF16 = 1, kEpiI32 = 2, kEpiGateUp = 3 };
 
 struct DecProblem {
     const int8_t* q;           // [M,K] codes
@@ -85,6 +89,7 @@ struct DecProblem {
     int64_t byte0;             // sum of R*K over the problems before this one
     int K;
     float beta;
+    float beta2;               // up projection's scale (kEpiGateUp)
     int epi;
 };
 
@@ -207,6 +212,7 @@ struct EpiConsts {
     int64_t N;
     int64_t R;
     float beta;
+    float beta2;
     int epi;
     __device__ __forceinline__ void load(const DecProblem& pr) {
         y = pr.y;
@@ -214,6 +220,7 @@ struct EpiConsts {
         N = pr.N;
         R = pr.R;
         beta = pr.beta;
+        beta2 = pr.beta2;
         epi = pr.epi;
     }
 };
@@ -234,6 +241,14 @@ __device__ __forceinline__ void store_output(const EpiConsts& e, int64_t idx, in
                 __fadd_rn(bf16_bits_to_float(__ldcg(e.residual + idx)), bf16_bits_to_float(b)));
         static_cast<uint16_t*>(e.y)[idx] = b;
     }
+}
+
+// z = relu2_mul(bf16(rescale(acc_gate)), bf16(rescale(acc_up))) of a gate/up pair.
+__device__ __forceinline__ void store_gate_up(const EpiConsts& e, int64_t idx, int acc_g, int acc_u,
+                                              const RecipDiv& s_x) {
+    const uint16_t a = float_to_bf16_bits(recip_div(__fmul_rn(__int2float_rn(acc_g), e.beta), s_x));
+    const uint16_t b = float_to_bf16_bits(recip_div(__fmul_rn(__int2float_rn(acc_u), e.beta2), s_x));
+    static_cast<uint16_t*>(e.y)[idx] = relu2_mul_one(a, b);
 }
 
 // Sum 4 per-lane partials over the warp (reduce-scatter: 6 shuffles).  On
@@ -455,14 +470,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
         if ((d.c + 1) * kDecChunk >= K || d.rows == 2) {  // the item ends its row(s)
 #pragma unroll
             for (int m = 0; m < MT; ++m) finish_acc(acc[m]);
+            // a gate/up pair takes the up total (bit pair i + 2) from the lane
+            // that holds it: 8 lanes up for half-warp rows, 16 for whole rows
+            const bool gu = ec.epi == kEpiGateUp;  // the same in the whole warp
             if (d.rows == 2) {
                 const int i = (lane >> 2) & 3;
                 const int64_t o = (int64_t)i * ec.R + d.r + (lane >> 4);
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     const int tot = half_reduce4(acc[m], lane);
-                    if ((lane & 3) == 0)
+                    if (gu) {
+                        const int up = __shfl_down_sync(0xffffffffu, tot, 8);
+                        if ((lane & 3) == 0 && i < 2)
+                            store_gate_up(ec, m * ec.N + o, (tot >> (2 * i)) - rsum[m],
+                                          (up >> (2 * i + 4)) - rsum[m], sx[m]);
+                    } else if ((lane & 3) == 0) {
                         store_output(ec, m * ec.N + o, (tot >> (2 * i)) - rsum[m], sx[m]);
+                    }
                 }
             } else {
                 const int i = lane >> 3;
@@ -470,8 +494,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_batch_kernel(
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     const int tot = warp_reduce4(acc[m], lane);
-                    if ((lane & 7) == 0)
+                    if (gu) {
+                        const int up = __shfl_down_sync(0xffffffffu, tot, 16);
+                        if ((lane & 7) == 0 && i < 2)
+                            store_gate_up(ec, m * ec.N + o, (tot >> (2 * i)) - rsum[m],
+                                          (up >> (2 * i + 4)) - rsum[m], sx[m]);
+                    } else if ((lane & 7) == 0) {
                         store_output(ec, m * ec.N + o, (tot >> (2 * i)) - rsum[m], sx[m]);
+                    }
                 }
             }
         }

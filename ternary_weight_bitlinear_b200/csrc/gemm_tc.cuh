@@ -83,6 +83,7 @@ struct TcArgs {
     int tiles_m;               // ceil(M / 128)
     int vec_ok;                // outputs of 32 consecutive rows can use 16-byte accesses
     int tma_store;             // bf16 y without residual: full 32 x 32 chunks leave by TMA store
+    float beta2;               // up projection's scale (kEpiGateUp)
     int64_t full_units;        // tiles processed whole; the rest as two N-halves each
     int64_t units;             // full_units + 2 * (tiles - full_units)
 };
@@ -182,6 +183,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
           "=r"(r[31])
         : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane (no wait).
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
@@ -497,6 +513,64 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kTcBN);
+            if (a.epi == kEpiGateUp) {
+                // gate columns [0, ucols/2) (bit pairs 0, 1), their up rows
+                // ucols/2 further on; this warp takes a quarter of the columns
+                const PairDiv sx2 = pair_div_init(sx.s, a.beta2);
+                const int gcb = half * (ucols / 4), gce = gcb + ucols / 4;
+#pragma unroll 1
+                for (int c0 = gcb; c0 < gce; c0 += 32) {
+                    uint32_t w[16];  // 32 bf16 outputs, two per word
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        uint32_t gv[16], uv[16];
+                        tmem_ld16_nowait(taddr + (uint32_t)(c0 + 16 * h2), gv);
+                        tmem_ld16_nowait(taddr + (uint32_t)(c0 + 16 * h2 + ucols / 2), uv);
+                        tmem_ld_wait();
+                        float yg[16], yu[16];
+                        scale16(gv, rsum, a.beta, sx, yg);
+                        scale16(uv, rsum, a.beta2, sx2, yu);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            w[8 * h2 + j] =
+                                (uint32_t)relu2_mul_one(float_to_bf16_bits(yg[2 * j]), float_to_bf16_bits(yu[2 * j])) |
+                                ((uint32_t)relu2_mul_one(float_to_bf16_bits(yg[2 * j + 1]),
+                                                         float_to_bf16_bits(yu[2 * j + 1])) << 16);
+                    }
+                    const int i = c0 >> lg;                                          // bit pair 0 or 1
+                    const int r = tn * kTcPackRows + rr0 + (c0 & ((1 << lg) - 1));  // first packed row
+                    const int valid = min(32, a.R - r);
+                    if (a.tma_store && valid == 32) {
+                        uint8_t* buf_out = stage + (nstore & 1) * kTcStageOut;
+                        if (lane == 0) bulk_wait_read_1();
+                        __syncwarp();
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            *reinterpret_cast<uint4*>(buf_out + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+                                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0)
+                            tma_store_2d(&tmap_y, smem_addr(buf_out), i * a.R + r, tm * kTcBM + q * 32);
+                        ++nstore;
+                    } else if (live && valid > 0) {
+                        uint16_t* zp = static_cast<uint16_t*>(a.y) + (int64_t)m * a.N + (int64_t)i * a.R + r;
+                        if (a.vec_ok && valid == 32) {
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                reinterpret_cast<uint4*>(zp)[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (j < valid) zp[j] = (uint16_t)(w[j >> 1] >> (16 * (j & 1)));
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(accempty_bar(buf));
+                continue;
+            }
 #pragma unroll 1
             for (int c0 = cb; c0 < ce; c0 += 32) {
                 uint32_t v[32];

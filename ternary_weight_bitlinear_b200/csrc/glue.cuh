@@ -12,12 +12,6 @@ namespace bl {
 
 constexpr int kGlueThreads = 256;
 
-__device__ __forceinline__ uint16_t relu2_mul_one(uint32_t a_bits, uint32_t b_bits) {
-    const float av = bf16_bits_to_float(a_bits);
-    const float ra = av > 0.0f ? av : 0.0f;
-    return float_to_bf16_bits(__fmul_rn(__fmul_rn(ra, ra), bf16_bits_to_float(b_bits)));
-}
-
 // One thread: 8 consecutive elements (one 16-byte vector), or the scalar tail.
 __global__ void __launch_bounds__(kGlueThreads) relu2_mul_kernel(const uint16_t* __restrict__ a,
                                                                  const uint16_t* __restrict__ b,

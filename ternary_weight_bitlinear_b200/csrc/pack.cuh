@@ -78,20 +78,29 @@ __device__ __forceinline__ uint32_t ternary_code(float w, float s_w) {
     return (uint32_t)(t + 1);
 }
 
+// Source of each bit pair (slot) of the packed rows: slot i of packed row r
+// takes row r of src[i], ternarised with the scale of ws[i].  One matrix:
+// src[i] = W + i*R*K (rows i*N/4 + r), one workspace.  A gate/up pair packed
+// as the concatenation [gate; up]: slots 0, 1 from the gate's two row halves
+// with the gate's scale, slots 2, 3 from the up projection's with its own.
+struct PackSlots {
+    const float* src[4];
+    const PackWorkspace* ws[4];
+};
+
 // One thread: 16 consecutive columns of one packed row (four source rows).
 __global__ void __launch_bounds__(kPackThreads) ternarize_pack_kernel(
-    const float* __restrict__ W, int64_t R, int64_t K, const PackWorkspace* __restrict__ ws,
-    uint8_t* __restrict__ P) {
+    const __grid_constant__ PackSlots sl, int64_t R, int64_t K, uint8_t* __restrict__ P) {
     pdl_wait();
     const int64_t cols16 = K >> 4;
     const int64_t idx = (int64_t)blockIdx.x * kPackThreads + threadIdx.x;
     if (idx >= R * cols16) return;
     const int64_t r = idx / cols16, c = idx - r * cols16;
-    const float s_w = __ldcg(&ws->s_w);
     uint32_t out[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float4* src = reinterpret_cast<const float4*>(W + (i * R + r) * K + c * 16);
+        const float s_w = __ldcg(&sl.ws[i]->s_w);
+        const float4* src = reinterpret_cast<const float4*>(sl.src[i] + r * K + c * 16);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
             const float4 f = __ldcg(src + v);

@@ -93,7 +93,9 @@ static_assert(kSkSmemBytes <= 227 * 1024, "shared memory budget");
 static_assert(kSkPBytes % 1024 == 0, "swizzle atoms stay 1024-aligned");
 static_assert(kSkMaxStages * (kSkPBytes + kSkKB * 16 * kSkBK) <= kSkRingBytes, "ring holds 8 stages at npad 16");
 static_assert(kSkDCol0 + 2 * kSkDBuf <= kSkTmemCols && kSkMaxTokens <= (int)kSkDBuf, "TMEM budget");
-static_assert(kSkThreads * 112 <= 65536, "register budget of one CTA per SM");
+// each of the four schedulers of an SM holds 16384 registers: with 18 warps one
+// scheduler holds 5, so at most 96 registers a thread (launch bounds below)
+static_assert((kSkThreads / 32 + 3) / 4 * 32 * 96 <= 16384, "register budget of one CTA per SM");
 
 struct SkProblem {
     const float* s_x;          // [M]
@@ -107,6 +109,7 @@ struct SkProblem {
     int tiles;                 // ceil(R / 32)
     int kst;                   // items per row tile: ceil(K / 512)
     float beta;
+    float beta2;               // up projection's scale (kEpiGateUp)
     int epi;
 };
 
@@ -202,17 +205,6 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// 16 consecutive 32-bit TMEM columns of this thread's lane (no wait).
-__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t* r) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32"
-        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-
 // 8 consecutive 32-bit TMEM columns of this thread's lane (no wait).
 __device__ __forceinline__ void tmem_ld8_nowait(uint32_t taddr, uint32_t (&r)[8]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
@@ -230,10 +222,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
           "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
           "r"(r[14]), "r"(r[15])
         : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld_wait() {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 // A (weights) from TMEM, B (tokens) from shared memory, D in TMEM.
@@ -320,6 +308,18 @@ __device__ __forceinline__ void sk_store(const SkProblem& pr, int m, int64_t n, 
                 __fadd_rn(bf16_bits_to_float(__ldcg(pr.residual + idx)), bf16_bits_to_float(bv)));
         static_cast<uint16_t*>(pr.y)[idx] = bv;
     }
+}
+
+// One output of a gate/up pair: relu2_mul(bf16 gate, bf16 up), both rescaled
+// through the token's reciprocal, each with its own weight scale.
+__device__ __forceinline__ void sk_store_gate_up(const SkProblem& pr, int m, int64_t n, int acc_g,
+                                                 int acc_u, float s_x, float s_rcp) {
+    const bool sfast = s_x >= 0x1p-40f && s_x <= 0x1p40f;
+    const bool fg = sfast && pr.beta >= 0x1p-40f && pr.beta <= 0x1p40f;
+    const bool fu = sfast && pr.beta2 >= 0x1p-40f && pr.beta2 <= 0x1p40f;
+    const uint16_t a = float_to_bf16_bits(sk_scale(acc_g, pr.beta, PairDiv{s_x, s_rcp, -s_x, fg}));
+    const uint16_t bb = float_to_bf16_bits(sk_scale(acc_u, pr.beta2, PairDiv{s_x, s_rcp, -s_x, fu}));
+    static_cast<uint16_t*>(pr.y)[(int64_t)m * pr.N + n] = relu2_mul_one(a, bb);
 }
 
 __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_constant__ SkBatch b) {
@@ -616,7 +616,19 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
                     uint32_t v8[8];
                     tmem_ld8_nowait(taddr + (uint32_t)cg, v8);
                     tmem_ld_wait();
-                    if (r < pr.R) {
+                    if (pr.epi == kEpiGateUp) {
+                        // the up row of bit pair bit + 2 sits 16 lanes up
+                        uint32_t u8[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) u8[k] = __shfl_down_sync(0xffffffffu, v8[k], 16);
+                        if (bit < 2 && r < pr.R) {
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                if (cg + k < cend)
+                                    sk_store_gate_up(pr, cg + k, n, (int)v8[k] - tok_rs[cg + k],
+                                                     (int)u8[k] - tok_rs[cg + k], tok_s[cg + k], tok_y[cg + k]);
+                        }
+                    } else if (r < pr.R) {
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
                             if (cg + k < cend)

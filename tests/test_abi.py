@@ -55,13 +55,14 @@ def test_workspace_sizes(L):
 
 
 def test_skinny_workspace_sizes(L):
-    """5..64 tokens add one split area (a flag and npad x 128 int32 per CTA)."""
+    """5..64 tokens add one split area (a counter and two blocks of 128 x npad
+    int32 per CTA)."""
     Q = B.bitlinear_quantized_batch_workspace_size
     assert Q(0) == Q(1) == Q(4) == Q(65) == Q(4096) == 0
     s5, s16, s17, s64 = Q(5), Q(16), Q(17), Q(64)
     assert 0 < s5 == s16 < s17 < s64           # npad 16, 16, 32, 64
     assert s64 - s16 == 3 * (s17 - s16)        # linear in npad
-    assert s64 >= 148 * 64 * 128 * 4          # room for every CTA of a B200
+    assert s64 >= 148 * 2 * 64 * 128 * 4      # room for every CTA of a B200
     own = 8 * 2560 + 2 * 256                  # codes + s_x + row sums (256-byte slices)
     assert B.bitlinear_forward_workspace_size(8, 2560, 640) == own + Q(8)
     assert B.bitlinear_forward_workspace_size(4, 2560, 640) == 4 * 2560 + 2 * 256
@@ -179,3 +180,32 @@ def test_binding_rejects_cpu_tensors():
     P = torch.zeros(32, 256, dtype=torch.uint8)
     with pytest.raises(TypeError):
         B.bitlinear_forward(x, P, 1.0)
+
+
+def test_gate_up_argument_checks(L):
+    sz = ctypes.c_size_t()
+    assert L.bitlinear_pack_gate_up_workspace_size(6912, 2560, ctypes.byref(sz)) == 0
+    assert sz.value > 0
+    assert L.bitlinear_pack_gate_up_workspace_size(7, 2560, ctypes.byref(sz)) == 2   # I odd
+    assert L.bitlinear_pack_gate_up_workspace_size(8, 24, ctypes.byref(sz)) == 2     # K % 16
+    ws = ctypes.c_size_t(1 << 20)
+    assert L.bitlinear_pack_gate_up(NULL, P16, 8, 32, P16, P16, P16, ws, NULL) == 1
+    assert L.bitlinear_pack_gate_up(P16, P16, 8, 32, P16, P16, P16, 0, NULL) == 5
+    assert L.bitlinear_pack_gate_up(P17, P16, 8, 32, P16, P16, P16, ws, NULL) == 3
+
+    def fgu(q=P16, s=P16, rs=P16, P=P16, M=2, K=32, I=8, z=P16, w=NULL, wb=0):
+        return L.bitlinear_forward_gate_up(q, s, rs, P, 1.0, 1.0, M, K, I, z, w, wb, NULL)
+
+    assert fgu(I=7) == 2
+    assert fgu(K=24) == 2
+    assert fgu(M=0) == 0                     # empty: nothing to do
+    assert fgu(z=NULL) == 1
+    assert fgu(P=P17) == 3
+    assert fgu(w=P17, wb=64) == 3
+
+
+def test_binding_exports_gate_up():
+    for n in ("bitlinear_pack_gate_up", "bitlinear_forward_gate_up",
+              "bitlinear_pack_gate_up_workspace_size"):
+        assert callable(getattr(B, n))
+

@@ -103,6 +103,12 @@ def special_rows(x):
     return x
 
 
+def guarded_quant(guard, M, K):
+    """Guarded code, scale and row-sum buffers for an [M,K] quantisation."""
+    return dict(q=guard.empty((M, K), torch.int8), s_x=guard.empty(M, torch.float32),
+                rowsum=guard.empty(M, torch.int32))
+
+
 @pytest.mark.parametrize("norm", [False, True])
 @pytest.mark.parametrize("M,K", [(1, 16), (3, 256), (4, 2560), (7, 6912), (64, 2560), (257, 272),
                                  # 1024+ rows: the register-resident kernels (two warps per
@@ -110,12 +116,6 @@ def special_rows(x):
                                  # shared-memory warp kernel
                                  (1024, 2560), (1031, 6912), (1100, 272), (1024, 2576),
                                  (1025, 7168), (1024, 8192), (1030, 8208)])
-def guarded_quant(guard, M, K):
-    """Guarded code, scale and row-sum buffers for an [M,K] quantisation."""
-    return dict(q=guard.empty((M, K), torch.int8), s_x=guard.empty(M, torch.float32),
-                rowsum=guard.empty(M, torch.int32))
-
-
 def test_act_quant_matches_oracle(M, K, norm, guard):
     x = special_rows(WL.activations(M, K, seed=M * 131 + K, outlier_frac=0.001))
     gain = WL.gain(K, seed=K) if norm else None
