@@ -21,6 +21,8 @@ forward           norm -> unpack -> quant -> matmul -> rescale
 relu2_mul         bf16(relu(a)^2 * b)
 residual_add      bf16(x + d)
 ffn_block         one FFN block of the 30-layer chain
+online_forward    weight scale + ternarise on this call, then forward (online QAT)
+ste_backward      linear backward on the dequantised operands (straight-through)
 """
 import ctypes
 import os
@@ -30,14 +32,25 @@ import numpy as np
 from . import build as _build
 
 _LIB = None
+_PARALLEL = False
+
+
+def set_parallel(on):
+    """Use the OpenMP build (matmul rows on all host cores, identical results)
+    for the calls that follow; the plain single-core build otherwise."""
+    global _LIB, _PARALLEL
+    if bool(on) != _PARALLEL:
+        _PARALLEL = bool(on)
+        _LIB = None
 
 
 def lib():
-    """Load (building first if needed) liboracle.so."""
+    """Load (building first if needed) liboracle.so, or liboracle_omp.so after
+    set_parallel(True)."""
     global _LIB
     if _LIB is None:
         path = _build.build()
-        L = ctypes.CDLL(path)
+        L = ctypes.CDLL(_build.LIB_OMP if _PARALLEL else path)
         P = ctypes.c_void_p
         i64 = ctypes.c_int64
         f32 = ctypes.c_float
@@ -75,6 +88,10 @@ def lib():
         L.ref_residual_add.restype = None
         L.ref_ffn_block.argtypes = [P, P, P, f32, P, f32, P, f32, P, f32, i64, i64, i64, P]
         L.ref_ffn_block.restype = ctypes.c_int
+        L.ref_online_forward.argtypes = [P, P, ctypes.c_int, f32, P, i64, i64, i64, P, P, P]
+        L.ref_online_forward.restype = ctypes.c_int
+        L.ref_ste_backward.argtypes = [P, P, P, P, f32, i64, i64, i64, P, P]
+        L.ref_ste_backward.restype = None
         _LIB = L
     return _LIB
 
@@ -243,3 +260,41 @@ def ffn_block(x, g_in, g_sub, eps, Pg, bg, Pu, bu, Pd, bd):
     if rc != 0:
         raise ValueError("ffn_block: bad shape")
     return out
+
+
+# --- online QAT -------------------------------------------------------------
+def online_forward(x, W, gain=None, eps=1e-5, norm=False):
+    """Forward with the weights quantised on this call from fp32 masters W
+    [N,K].  Returns dict(y=fp32 [M,N], beta, t=int8 [N,K])."""
+    x = _c(x, np.uint16)
+    W = _c(W, np.float32)
+    M, K = x.shape
+    N = W.shape[0]
+    g = None if gain is None else _c(gain, np.uint16)
+    y = np.empty((M, N), np.float32)
+    beta = ctypes.c_float()
+    t = np.empty((N, K), np.int8)
+    rc = lib().ref_online_forward(_p(x), _p(g), 1 if norm else 0, ctypes.c_float(eps), _p(W), M,
+                                  K, N, _p(y), ctypes.byref(beta), _p(t))
+    if rc != 0:
+        raise ValueError("online_forward: bad shape")
+    return dict(y=y, beta=float(np.float32(beta.value)), t=t)
+
+
+def ste_backward(gy, q, s_x, t, beta):
+    """Gradients (gx [M,K], gw [N,K], float64) of the layer under the
+    straight-through estimator, from the output gradient gy [M,N] (fp32), the
+    forward's codes q [M,K] and scales s_x [M], and the ternary weights t
+    [N,K] with their absmean beta."""
+    gy = _c(gy, np.float32)
+    q = _c(q, np.int8)
+    s_x = _c(s_x, np.float32)
+    t = _c(t, np.int8)
+    M, N = gy.shape
+    K = q.shape[1]
+    gx = np.empty((M, K), np.float64)
+    gw = np.empty((N, K), np.float64)
+    lib().ref_ste_backward(_p(gy), _p(q), _p(s_x), _p(t), ctypes.c_float(beta), M, K, N, _p(gx),
+                           _p(gw))
+    return gx, gw
+

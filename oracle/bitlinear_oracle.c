@@ -328,6 +328,10 @@ void ref_ternary_matmul(const int8_t* q, const int8_t* t, int64_t M, int64_t K, 
                         int32_t* acc) {
     for (int64_t m = 0; m < M; ++m) {
         const int8_t* qr = q + m * K;
+        /* the outputs of a row are independent exact integer sums: the
+         * OpenMP build (liboracle_omp.so) computes them on all host cores,
+         * the plain build one after another, with identical results */
+#pragma omp parallel for schedule(static)
         for (int64_t n = 0; n < N; ++n) {
             const int8_t* tr = t + n * K;
             int32_t s = 0;
@@ -440,4 +444,73 @@ int ref_ffn_block(const uint16_t* x, const uint16_t* g_in, const uint16_t* g_sub
 done:
     free(yf); free(a); free(b); free(z); free(d);
     return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Online quantisation-aware training.  "Transformers 实战 BitNet 1.58 位量化"
+ * walkthrough: "量化器参数：BitNetQuantConfig 详解" (AutoBitLinear with
+ * quantization_mode "online" quantises the weights on every forward through
+ * WeightQuant) and "BitLinear 的三步量化" (steps 1-3, and the straight-through
+ * estimator of both quantisers' backward).                                 */
+/* ------------------------------------------------------------------------ */
+
+/* The online forward: the weight scale and the ternary weights are derived
+ * from the fp32 master weights W [N,K] on this call (steps 1-2), then the
+ * forward is the BitLinear forward of ref_forward on them.  beta_out (the
+ * absmean) and t_out [N,K] are optional outputs.  Returns 0, or -1 on a bad
+ * shape or allocation failure.                                             */
+int ref_online_forward(const uint16_t* x, const uint16_t* gain, int use_norm, float eps,
+                       const float* W, int64_t M, int64_t K, int64_t N, float* y,
+                       float* beta_out, int8_t* t_out) {
+    if (M < 0 || K <= 0 || N <= 0 || N % 4 != 0) return -1;
+    int8_t* t = (int8_t*)malloc((size_t)(N * K));
+    uint8_t* P = (uint8_t*)malloc((size_t)(N / 4 * K));
+    int rc = -1;
+    if (!t || !P) goto done;
+    float beta = ref_weight_scale(W, N, K);
+    ref_ternarize(W, N * K, beta, t);
+    if (ref_pack(t, N, K, P)) goto done;
+    if (ref_forward(x, gain, use_norm, eps, P, beta, M, K, N, y, NULL, NULL, NULL)) goto done;
+    if (beta_out) *beta_out = beta;
+    if (t_out) memcpy(t_out, t, (size_t)(N * K));
+    rc = 0;
+done:
+    free(t); free(P);
+    return rc;
+}
+
+/* The backward of the layer under the straight-through estimator: both
+ * quantisers pass the gradient through unchanged (grad_input = grad_output),
+ * so the gradients are those of the linear layer on the dequantised operands
+ * the forward multiplied (step 2: weight = round-and-clamp(W * scale) / scale;
+ * step 3: activation = round-and-clamp(x * scale) / scale):
+ *   W_q[n,k] = RN32( t[n,k] / s_w ),  s_w = RN32(1 / beta)
+ *   x_q[m,k] = RN32( q[m,k] / s_x[m] )
+ *   gx[m,k]  = sum_n gy[m,n] * W_q[n,k]      (grad of the input)
+ *   gw[n,k]  = sum_m gy[m,n] * x_q[m,k]      (grad of the master weight)
+ * gy [M,N] binary32; the products of two binary32 values are exact in
+ * binary64 and the sums are taken in binary64 in index order.              */
+void ref_ste_backward(const float* gy, const int8_t* q, const float* s_x, const int8_t* t,
+                      float beta, int64_t M, int64_t K, int64_t N, double* gx, double* gw) {
+    float s_w = 1.0f / beta;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                float wq = (float)t[n * K + k] / s_w;
+                s += (double)gy[m * N + n] * (double)wq;
+            }
+            gx[m * K + k] = s;
+        }
+    }
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t m = 0; m < M; ++m) {
+                float xq = (float)q[m * K + k] / s_x[m];
+                s += (double)gy[m * N + n] * (double)xq;
+            }
+            gw[n * K + k] = s;
+        }
+    }
 }

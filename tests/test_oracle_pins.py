@@ -526,3 +526,112 @@ def test_ffn_block_equals_its_steps(O):
     z = O.relu2_mul(a, b)
     d = O.f32_to_bf16(O.forward(z, Pd, bd, gain=g2, norm=True)["y"])
     np.testing.assert_array_equal(out, O.residual_add(x, d))
+
+
+def test_openmp_build_gives_identical_results(O):
+    """The oracle's OpenMP build (matmul rows on all host cores, used for the
+    CPU baseline) returns the plain build's results bit for bit."""
+    rng = np.random.default_rng(77)
+    W = (rng.standard_normal((256, 512)) * 0.02).astype(np.float32)
+    P, beta = O.pack_master(W)
+    x = bf16(rng.standard_normal((5, 512)))
+    g = bf16(rng.uniform(0.5, 1.5, 512))
+    ref = O.forward(x, P, beta, gain=g, eps=1e-5, norm=True)
+    try:
+        O.set_parallel(True)
+        par = O.forward(x, P, beta, gain=g, eps=1e-5, norm=True)
+    finally:
+        O.set_parallel(False)
+    assert (par["acc"] == ref["acc"]).all()
+    assert (par["y"].view(np.uint32) == ref["y"].view(np.uint32)).all()
+
+
+# --------------------------------------------------------------------------
+# Online QAT: forward with on-the-fly ternarisation, straight-through backward
+# --------------------------------------------------------------------------
+def test_online_forward_reproduces_the_hand_example(O):
+    """The online forward starts from the fp32 masters: on the hand-worked
+    example it must land on the hand-derived beta, ternary weights and y."""
+    g = load_golden("hand_example_4x8.txt")
+    W = np.array([[parse_float(v) for v in g["W_row%d" % i]] for i in range(4)], np.float32)
+    t_exp = np.array([[int(v) for v in g["t_row%d" % i]] for i in range(4)], np.int8)
+    x = np.array([[parse_float(v) for v in g["x_row%d" % i]] for i in range(4)], np.float32)
+    y_exp = np.array([[rn32_of_fraction(Fraction(v)) for v in g["y_row%d" % i]]
+                      for i in range(4)], np.float32)
+    out = O.online_forward(bf16(x), W)
+    assert out["beta"] == parse_float(g["beta"][0])
+    np.testing.assert_array_equal(out["t"], t_exp)
+    np.testing.assert_array_equal(out["y"].view(np.uint32), y_exp.view(np.uint32))
+
+
+def test_online_forward_is_the_forward_of_the_packed_masters(O):
+    rng = np.random.default_rng(90)
+    W = (rng.standard_normal((64, 96)) * 0.02).astype(np.float32)
+    x = bf16(rng.standard_normal((3, 96)))
+    gain = bf16(rng.uniform(0.5, 1.5, 96))
+    P, beta = O.pack_master(W)
+    for norm in (False, True):
+        on = O.online_forward(x, W, gain=gain, eps=1e-5, norm=norm)
+        ref = O.forward(x, P, beta, gain=gain, eps=1e-5, norm=norm)
+        assert on["beta"] == beta
+        assert (on["y"].view(np.uint32) == ref["y"].view(np.uint32)).all()
+
+
+def _dequantised(O, q, s_x, t, beta):
+    """W_q = RN32(t / RN32(1/beta)), x_q = RN32(q / s_x), by numpy binary32."""
+    s_w = np.float32(1.0) / np.float32(beta)
+    W_q = (t.astype(np.float32) / s_w).astype(np.float32)
+    x_q = (q.astype(np.float32) / s_x[:, None].astype(np.float32)).astype(np.float32)
+    return W_q, x_q
+
+
+def test_ste_backward_one_hot_gradients(O):
+    """A one-hot output gradient selects one row of each dequantised operand:
+    gx[m0] = W_q[n0] and gw[n0] = x_q[m0] exactly, zeros elsewhere."""
+    rng = np.random.default_rng(91)
+    M, K, N = 3, 40, 8
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    beta = O.weight_scale(W)
+    t = O.ternarize(W, beta)
+    q, s, _ = O.quantize_input(bf16(rng.standard_normal((M, K)) * 3))
+    W_q, x_q = _dequantised(O, q, s, t, beta)
+    for m0, n0 in ((0, 0), (2, 5), (1, 7)):
+        gy = np.zeros((M, N), np.float32)
+        gy[m0, n0] = 1.0
+        gx, gw = O.ste_backward(gy, q, s, t, beta)
+        exp_gx = np.zeros((M, K))
+        exp_gx[m0] = W_q[n0]
+        exp_gw = np.zeros((N, K))
+        exp_gw[n0] = x_q[m0]
+        np.testing.assert_array_equal(gx, exp_gx)
+        np.testing.assert_array_equal(gw, exp_gw)
+    # the dequantised weight magnitude is RN32(1 / RN32(1 / beta)): beta give or take an ulp
+    mag = np.abs(W_q[W_q != 0])
+    assert np.all(mag == mag[0]) and abs(float(mag[0]) - beta) <= float(np.spacing(np.float32(beta)))
+
+
+def test_ste_backward_against_exact_rationals(O):
+    """Tiny shapes: the binary64 sums against exact rational sums of the same
+    binary32 products, within the rounding bound of n binary64 additions."""
+    rng = np.random.default_rng(92)
+    M, K, N = 4, 6, 8
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    beta = O.weight_scale(W)
+    t = O.ternarize(W, beta)
+    q, s, _ = O.quantize_input(bf16(rng.standard_normal((M, K))))
+    gy = rng.standard_normal((M, N)).astype(np.float32)
+    gx, gw = O.ste_backward(gy, q, s, t, beta)
+    W_q, x_q = _dequantised(O, q, s, t, beta)
+    u = 2.0 ** -53
+    for m in range(M):
+        for k in range(K):
+            terms = [Fraction(float(gy[m, n])) * Fraction(float(W_q[n, k])) for n in range(N)]
+            exact = sum(terms, Fraction(0))
+            bound = N * u * float(sum(abs(v) for v in terms))
+            assert abs(Fraction(gx[m, k]) - exact) <= Fraction(bound) + Fraction(1, 10 ** 300)
+    for n in range(N):
+        for k in range(K):
+            terms = [Fraction(float(gy[m, n])) * Fraction(float(x_q[m, k])) for m in range(M)]
+            exact = sum(terms, Fraction(0))
+            bound = M * u * float(sum(abs(v) for v in terms))
+            assert abs(Fraction(gw[n, k]) - exact) <= Fraction(bound) + Fraction(1, 10 ** 300)
