@@ -267,6 +267,51 @@ bl_status bitlinear_forward_gate_up(const int8_t* q, const float* s_x, const int
                                     int64_t K, int64_t I, uint16_t* z, void* workspace,
                                     size_t workspace_bytes, void* stream);
 
+/* ---- quantisation-aware training (online quantisation, STE backward) ---- */
+
+/* Workspace bitlinear_forward_online needs: the absmean partial sums and, for
+ * 5 <= M <= 64, the split-tile area of the 5..64-token kernel. */
+bl_status bitlinear_forward_online_workspace_size(int64_t M, int64_t K, int64_t N,
+                                                  size_t* bytes);
+
+/* The training-time forward of a BitLinear whose weights are quantised on
+ * every call ([BG] "量化器参数：BitNetQuantConfig 详解": AutoBitLinear with
+ * quantization_mode "online"; [BG] "BitLinear 的三步量化" steps 1-3): the
+ * absmean scale and the ternary weights come from the fp32 master weights on
+ * this call, exactly as bitlinear_pack computes them, and the forward is the
+ * inference forward on them (bit for bit bitlinear_pack followed by
+ * bitlinear_forward).  All asynchronous: the scale stays on the device.
+ *   x, gain, eps, y, y_dtype  as for bitlinear_forward (x may be NULL when M == 0).
+ *   W        device fp32 [N,K] master weights.
+ *   P        device uint8 [N/4,K] output: the packed ternary weights.
+ *   beta     device float[1] output: the absmean scale (input of the backward).
+ *   q, s_x, rowsum  device outputs [M,K] int8, [M] fp32, [M] int32: the
+ *            quantised activations (inputs of the backward).
+ *   workspace  device, >= bitlinear_forward_online_workspace_size bytes. */
+bl_status bitlinear_forward_online(const uint16_t* x, const uint16_t* gain, float eps,
+                                   const float* W, int64_t M, int64_t K, int64_t N, void* y,
+                                   bl_out_dtype y_dtype, uint8_t* P, float* beta, int8_t* q,
+                                   float* s_x, int32_t* rowsum, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/* The backward of that layer under the straight-through estimator ([BG]
+ * "BitLinear 的三步量化": both quantisers pass the gradient through unchanged),
+ * i.e. the linear layer's backward on the dequantised operands:
+ *   W_q[n,k] = RN32(t[n,k] / RN32(1/beta)),  x_q[m,k] = RN32(q[m,k] / s_x[m]),
+ *   grad_x[m,k] = sum_n grad_y[m,n] W_q[n,k],
+ *   grad_w[n,k] = sum_m grad_y[m,n] x_q[m,k]   (the master weights' gradient).
+ * Sums in binary32, each product added with one fused multiply-add; the order
+ * of the additions is not specified, so results agree with the exact sums to
+ * within n * 2^-24 * sum |terms| (n = N for grad_x, M for grad_w).
+ *   grad_y  device fp32 [M,N].
+ *   q, s_x  device, from bitlinear_forward_online (needed for grad_w).
+ *   P, beta device, from bitlinear_forward_online (needed for grad_x).
+ *   grad_x  device fp32 [M,K] output, or NULL to skip it.
+ *   grad_w  device fp32 [N,K] output, or NULL to skip it (not both NULL). */
+bl_status bitlinear_backward_ste(const float* grad_y, const int8_t* q, const float* s_x,
+                                 const uint8_t* P, const float* beta, int64_t M, int64_t K,
+                                 int64_t N, float* grad_x, float* grad_w, void* stream);
+
 /* ---- forward without any caller-provided memory besides inputs and outputs -- */
 
 /* Size of the library's fixed device scratch used by bitlinear_forward_noalloc. */

@@ -9,6 +9,8 @@ from .bitlinear import (BL_MAX_K, BL_OUT_BF16, BL_OUT_F32, BitLinearError, LIB_P
                         bitlinear_forward_batch_workspace_size, bitlinear_forward_quantized,
                         bitlinear_forward_quantized_batch, bitlinear_forward_gate_up,
                         bitlinear_pack_gate_up, bitlinear_pack_gate_up_workspace_size,
+                        bitlinear_forward_online, bitlinear_forward_online_workspace_size,
+                        bitlinear_backward_ste,
                         make_batch,
                         make_quantized_batch,
                         bitlinear_forward_workspace_size, bitlinear_pack,

@@ -42,6 +42,10 @@ SIGNATURES = {
     "bitlinear_pack_gate_up": ([_P, _P, _I64, _I64, _P, _P, _P, _SZ, _P], _INT),
     "bitlinear_forward_gate_up": ([_P, _P, _P, _P, _F32, _F32, _I64, _I64, _I64, _P, _P, _SZ, _P],
                                   _INT),
+    "bitlinear_forward_online_workspace_size": ([_I64, _I64, _I64, ctypes.POINTER(_SZ)], _INT),
+    "bitlinear_forward_online": ([_P, _P, _F32, _P, _I64, _I64, _I64, _P, _INT, _P, _P, _P, _P, _P,
+                                  _P, _SZ, _P], _INT),
+    "bitlinear_backward_ste": ([_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P], _INT),
     "bitlinear_forward_noalloc": ([_P, _P, _F32, _P, _F32, _I64, _I64, _I64, _P, _INT, _P], _INT),
     "bitlinear_device_status": ([_P], _INT),
     "bitlinear_selftest_wait_timeout": ([_I64, _P], _INT),
@@ -343,6 +347,52 @@ def bitlinear_forward_gate_up(q, s_x, rowsum, P2, beta_gate, beta_up, out=None, 
         _ptr(q), _ptr(s_x), _ptr(rowsum), _ptr(P2), float(beta_gate), float(beta_up), M, K, I,
         _ptr(z), _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream)))
     return z
+
+
+def bitlinear_forward_online_workspace_size(M, K, N):
+    n = ctypes.c_size_t()
+    _check("bitlinear_forward_online_workspace_size",
+           lib().bitlinear_forward_online_workspace_size(M, K, N, ctypes.byref(n)))
+    return n.value
+
+
+def bitlinear_forward_online(x, W, gain=None, eps=1e-5, out_dtype=torch.bfloat16, out=None,
+                             workspace=None, stream=None):
+    """Training forward from fp32 masters W [N,K]: returns (y, saved) where
+    saved = dict(P, beta (device fp32 [1]), q, s_x, rowsum) feeds the backward."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(W, torch.float32, "W", 2)
+    if gain is not None:
+        _need(gain, torch.bfloat16, "gain", 1)
+    M, K = x.shape
+    N = W.shape[0]
+    dev = x.device
+    y = torch.empty((M, N), dtype=out_dtype, device=dev) if out is None else out
+    saved = dict(P=torch.empty((N // 4, K), dtype=torch.uint8, device=dev),
+                 beta=torch.empty(1, dtype=torch.float32, device=dev),
+                 q=torch.empty((M, K), dtype=torch.int8, device=dev),
+                 s_x=torch.empty(M, dtype=torch.float32, device=dev),
+                 rowsum=torch.empty(M, dtype=torch.int32, device=dev))
+    ws = _workspace(bitlinear_forward_online_workspace_size(M, K, N), dev) \
+        if workspace is None else workspace
+    _check("bitlinear_forward_online", lib().bitlinear_forward_online(
+        _ptr(x), _ptr(gain), eps, _ptr(W), M, K, N, _ptr(y), _out_code(y.dtype), _ptr(saved["P"]),
+        _ptr(saved["beta"]), _ptr(saved["q"]), _ptr(saved["s_x"]), _ptr(saved["rowsum"]),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return y, saved
+
+
+def bitlinear_backward_ste(grad_y, saved, K, grad_x=True, grad_w=True, stream=None):
+    """Straight-through backward: (grad_x fp32 [M,K] or None, grad_w fp32 [N,K] or None)."""
+    _need(grad_y, torch.float32, "grad_y", 2)
+    M, N = grad_y.shape
+    dev = grad_y.device
+    gx = torch.empty((M, K), dtype=torch.float32, device=dev) if grad_x else None
+    gw = torch.empty((N, K), dtype=torch.float32, device=dev) if grad_w else None
+    _check("bitlinear_backward_ste", lib().bitlinear_backward_ste(
+        _ptr(grad_y), _ptr(saved["q"]), _ptr(saved["s_x"]), _ptr(saved["P"]), _ptr(saved["beta"]),
+        M, K, N, _ptr(gx), _ptr(gw), _stream(stream)))
+    return gx, gw
 
 
 def bitlinear_selftest_wait_timeout(limit_ns, stream=None):

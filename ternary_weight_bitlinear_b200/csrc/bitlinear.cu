@@ -21,6 +21,7 @@
 #include "pack.cuh"
 #include "quant.cuh"
 #include "skinny.cuh"
+#include "ste.cuh"
 
 namespace {
 
@@ -234,6 +235,7 @@ struct DecodeJob {
     float beta;
     int epi;
     float beta2 = 0.0f;  // kEpiGateUp: the up projection's scale
+    const float* beta_dev = nullptr;  // beta read from device memory instead (online forward)
     // packed rows of P: N/4, or N/2 for a gate/up pair (N = the pair's I outputs)
     int64_t packed_rows() const { return epi == kEpiGateUp ? N / 2 : N / 4; }
 };
@@ -270,6 +272,7 @@ bl_status launch_decode_cap(const DecodeJob* jobs, int count, int mt, int dev,
         p.K = (int)jobs[i].K;
         p.beta = jobs[i].beta;
         p.beta2 = jobs[i].beta2;
+        p.beta_dev = jobs[i].beta_dev;
         p.epi = jobs[i].epi;
         total += p.R * p.K;
         rows += p.R;
@@ -372,6 +375,7 @@ bl_status run_gemm(const DecodeJob& j, int64_t M, int dev, const DeviceInfo& inf
     a.residual = residual;
     a.beta = j.beta;
     a.beta2 = j.beta2;
+    a.beta_dev = j.beta_dev;
     a.epi = epi;
     a.M = (int)M;
     a.K = (int)K;
@@ -450,6 +454,7 @@ bl_status run_skinny(const DecodeJob* jobs, int count, int64_t M, void* ws, size
             p.kst = (p.K + kSkItemK - 1) / kSkItemK;
             p.beta = j.beta;
             p.beta2 = j.beta2;
+            p.beta_dev = j.beta_dev;
             p.epi = j.epi;
             p.item0 = items;
             items += (int64_t)p.tiles * p.kst;
@@ -821,6 +826,90 @@ bl_status bitlinear_forward_gate_up(const int8_t* q, const float* s_x, const int
     j.beta2 = beta_up;
     return run_job(j, M, dev, info, static_cast<cudaStream_t>(stream), workspace,
                    workspace ? workspace_bytes : 0);
+}
+
+bl_status bitlinear_forward_online_workspace_size(int64_t M, int64_t K, int64_t N,
+                                                  size_t* bytes) {
+    if (!bytes) return BL_ERR_NULL;
+    bl_status st = check_shape(M, K, N);
+    if (st != BL_OK) return st;
+    *bytes = (size_t)(round_up((int64_t)sizeof(PackWorkspace), 256) + sk_ws_bytes(M));
+    return BL_OK;
+}
+
+bl_status bitlinear_forward_online(const uint16_t* x, const uint16_t* gain, float eps,
+                                   const float* W, int64_t M, int64_t K, int64_t N, void* y,
+                                   bl_out_dtype y_dtype, uint8_t* P, float* beta, int8_t* q,
+                                   float* s_x, int32_t* rowsum, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    size_t need = 0;
+    bl_status st = bitlinear_forward_online_workspace_size(M, K, N, &need);
+    if (st != BL_OK) return st;
+    const int epi = epi_of(y_dtype);
+    if (epi < 0) return BL_ERR_DTYPE;
+    if (!W || !P || !beta) return BL_ERR_NULL;
+    if (M > 0 && (!x || !y || !q || !s_x || !rowsum)) return BL_ERR_NULL;
+    if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(W) || !aligned16(P) || !aligned16(workspace) || (x && !aligned16(x)) ||
+        (y && !aligned16(y)) || (q && !aligned16(q)) || (gain && !aligned16(gain)))
+        return BL_ERR_ALIGN;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the weight scale and the packed ternary weights of this call
+    PackWorkspace* pw = static_cast<PackWorkspace*>(workspace);
+    const int64_t n = N * K, R = N / 4, work = R * (K / 16);
+    if ((st = launch(absmean_partial_kernel, dim3(kPackPartials), dim3(kPackThreads), 0, s, W, n,
+                     pw)) != BL_OK)
+        return st;
+    if ((st = launch(absmean_finalize_kernel, dim3(1), dim3(32), 0, s, n, kPackPartials, pw,
+                     beta)) != BL_OK)
+        return st;
+    PackSlots sl;
+    for (int i = 0; i < 4; ++i) {
+        sl.src[i] = W + (int64_t)i * R * K;
+        sl.ws[i] = pw;
+    }
+    if ((st = launch(ternarize_pack_kernel,
+                     dim3((unsigned)((work + kPackThreads - 1) / kPackThreads)),
+                     dim3(kPackThreads), 0, s, sl, R, K, P)) != BL_OK)
+        return st;
+    if (M == 0) return BL_OK;
+    // then the forward on them, the rescale reading beta from device memory
+    QuantProblem qp = {x, gain, q, s_x, rowsum, (int)K};
+    if ((st = run_quant(&qp, 1, M, eps, dev, info, s)) != BL_OK) return st;
+    DecodeJob j = {q, s_x, rowsum, P, y, nullptr, K, N, 1.0f, epi};
+    j.beta_dev = beta;
+    const int64_t own = round_up((int64_t)sizeof(PackWorkspace), 256);
+    return run_job(j, M, dev, info, s, static_cast<char*>(workspace) + own,
+                   workspace_bytes - (size_t)own);
+}
+
+bl_status bitlinear_backward_ste(const float* grad_y, const int8_t* q, const float* s_x,
+                                 const uint8_t* P, const float* beta, int64_t M, int64_t K,
+                                 int64_t N, float* grad_x, float* grad_w, void* stream) {
+    bl_status st = check_shape(M, K, N);
+    if (st != BL_OK) return st;
+    if (M == 0) return BL_OK;
+    if (!grad_y || !beta || (!grad_x && !grad_w)) return BL_ERR_NULL;
+    if ((grad_x && !P) || (grad_w && (!q || !s_x))) return BL_ERR_NULL;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned tk = (unsigned)((K + kSteTile - 1) / kSteTile);
+    if (grad_x &&
+        (st = launch(ste_grad_input_kernel,
+                     dim3(tk, (unsigned)((M + kSteTile - 1) / kSteTile)), dim3(kSteThreads), 0, s,
+                     grad_y, P, beta, M, K, N, grad_x)) != BL_OK)
+        return st;
+    if (grad_w &&
+        (st = launch(ste_grad_weight_kernel,
+                     dim3(tk, (unsigned)((N + kSteTile - 1) / kSteTile)), dim3(kSteThreads), 0, s,
+                     grad_y, q, s_x, M, K, N, grad_w)) != BL_OK)
+        return st;
+    return BL_OK;
 }
 
 bl_status bitlinear_quantized_batch_workspace_size(int64_t M, size_t* bytes) {

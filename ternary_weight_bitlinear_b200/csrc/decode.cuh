@@ -91,6 +91,7 @@ struct DecProblem {
     float beta;
     float beta2;               // up projection's scale (kEpiGateUp)
     int epi;
+    const float* beta_dev;     // when set: beta is read from device memory (after the grid wait)
 };
 
 template <int CAP>
@@ -219,7 +220,7 @@ struct EpiConsts {
         residual = pr.residual;
         N = pr.N;
         R = pr.R;
-        beta = pr.beta;
+        beta = pr.beta_dev ? __ldcg(pr.beta_dev) : pr.beta;
         beta2 = pr.beta2;
         epi = pr.epi;
     }

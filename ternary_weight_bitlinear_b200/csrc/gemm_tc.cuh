@@ -84,6 +84,7 @@ struct TcArgs {
     int vec_ok;                // outputs of 32 consecutive rows can use 16-byte accesses
     int tma_store;             // bf16 y without residual: full 32 x 32 chunks leave by TMA store
     float beta2;               // up projection's scale (kEpiGateUp)
+    const float* beta_dev;     // when set: beta is read from device memory
     int64_t full_units;        // tiles processed whole; the rest as two N-halves each
     int64_t units;             // full_units + 2 * (tiles - full_units)
 };
@@ -271,15 +272,16 @@ __device__ __forceinline__ float tc_scale(int acc, float beta, const PairDiv& s_
 
 // Store 32 consecutive outputs y[m, n0 .. n0+31] of one token (scalar path:
 // only rows < R, i.e. n0 + j with j < valid).
-__device__ __forceinline__ void tc_store_row32(const TcArgs& a, int64_t base, const uint32_t (&v)[32], int rsum,
-                               const PairDiv& s_x, int valid) {
+__device__ __forceinline__ void tc_store_row32(const TcArgs& a, float beta, int64_t base,
+                                               const uint32_t (&v)[32], int rsum, const PairDiv& s_x,
+                                               int valid) {
     if (a.vec_ok && valid == 32) {
         if (a.epi == kEpiBF16) {
             uint32_t w[16];
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
                 float y[16];
-                scale16(v + 16 * g, rsum, a.beta, s_x, y);
+                scale16(v + 16 * g, rsum, beta, s_x, y);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) w[8 * g + j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
             }
@@ -306,7 +308,7 @@ __device__ __forceinline__ void tc_store_row32(const TcArgs& a, int64_t base, co
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
                 float y[16];
-                scale16(v + 16 * g, rsum, a.beta, s_x, y);
+                scale16(v + 16 * g, rsum, beta, s_x, y);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     yp[4 * g + c] = make_uint4(__float_as_uint(y[4 * c]), __float_as_uint(y[4 * c + 1]),
@@ -329,9 +331,9 @@ __device__ __forceinline__ void tc_store_row32(const TcArgs& a, int64_t base, co
         if (a.epi == kEpiI32) {
             static_cast<int32_t*>(a.y)[idx] = acc;
         } else if (a.epi == kEpiF32) {
-            static_cast<float*>(a.y)[idx] = tc_scale(acc, a.beta, s_x);
+            static_cast<float*>(a.y)[idx] = tc_scale(acc, beta, s_x);
         } else {
-            uint16_t b = float_to_bf16_bits(tc_scale(acc, a.beta, s_x));
+            uint16_t b = float_to_bf16_bits(tc_scale(acc, beta, s_x));
             if (a.residual)
                 b = float_to_bf16_bits(
                     __fadd_rn(bf16_bits_to_float(__ldcg(a.residual + idx)), bf16_bits_to_float(b)));
@@ -488,6 +490,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
         }
     } else {
         // ---------------- epilogue: one token per thread ----------------
+        const float beta = a.beta_dev ? __ldcg(a.beta_dev) : a.beta;
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
         const int half = (warp - kTcEpiWarp0) >> 2;  // which 128 of the 256 columns
         // this warp's two staging buffers (64-byte rows, 64-byte swizzle: chunk c
@@ -507,7 +510,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
             const int buf = (int)(tl & 1);
             const int m = tm * kTcBM + q * 32 + lane;  // this thread's token
             const bool live = m < a.M;
-            const PairDiv sx = pair_div_init((live && a.epi != kEpiI32) ? __ldcg(a.s_x + m) : 1.0f, a.beta);
+            const PairDiv sx = pair_div_init((live && a.epi != kEpiI32) ? __ldcg(a.s_x + m) : 1.0f, beta);
             const int rsum = live ? __ldcg(a.rowsum + m) : 0;
             const bool got = mbar_wait(accfull_bar(buf), (tl >> 1) & 1u);
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -528,7 +531,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
                         tmem_ld16_nowait(taddr + (uint32_t)(c0 + 16 * h2 + ucols / 2), uv);
                         tmem_ld_wait();
                         float yg[16], yu[16];
-                        scale16(gv, rsum, a.beta, sx, yg);
+                        scale16(gv, rsum, beta, sx, yg);
                         scale16(uv, rsum, a.beta2, sx2, yu);
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
@@ -584,7 +587,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
 #pragma unroll
                     for (int g = 0; g < 2; ++g) {
                         float y[16];
-                        scale16(v + 16 * g, rsum, a.beta, sx, y);
+                        scale16(v + 16 * g, rsum, beta, sx, y);
 #pragma unroll
                         for (int j = 0; j < 8; ++j) w[8 * g + j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
                     }
@@ -601,7 +604,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
                         tma_store_2d(&tmap_y, smem_addr(buf_out), i * a.R + r, tm * kTcBM + q * 32);
                     ++nstore;
                 } else if (live && valid > 0) {
-                    tc_store_row32(a, (int64_t)m * a.N + (int64_t)i * a.R + r, v, rsum, sx, valid);
+                    tc_store_row32(a, beta, (int64_t)m * a.N + (int64_t)i * a.R + r, v, rsum, sx, valid);
                 }
             }
             tc_fence_before();

@@ -111,6 +111,7 @@ struct SkProblem {
     float beta;
     float beta2;               // up projection's scale (kEpiGateUp)
     int epi;
+    const float* beta_dev;     // when set: beta is read from device memory
 };
 
 struct alignas(64) SkBatch {
@@ -532,7 +533,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
         while (item < i1 && ok) {
             // the part of (cur.p, cur.tile) inside this CTA's share; the
             // problem's constants are copied to registers once per part
-            const SkProblem pr = b.p[cur.p];
+            SkProblem pr = b.p[cur.p];
+            if (pr.beta_dev) pr.beta = __ldcg(pr.beta_dev);
             if (staged != cur.p) {  // this problem's token scales and row sums, once
                 sk_epi_sync();
                 if (et < b.M) {

@@ -209,3 +209,36 @@ def test_binding_exports_gate_up():
               "bitlinear_pack_gate_up_workspace_size"):
         assert callable(getattr(B, n))
 
+
+
+def test_online_and_backward_argument_checks(L):
+    sz = ctypes.c_size_t()
+    assert L.bitlinear_forward_online_workspace_size(8, 256, 128, ctypes.byref(sz)) == 0
+    small = sz.value
+    assert small > 0
+    assert L.bitlinear_forward_online_workspace_size(1, 256, 128, ctypes.byref(sz)) == 0
+    assert sz.value < small                      # no split area below five tokens
+    assert L.bitlinear_forward_online_workspace_size(1, 250, 128, ctypes.byref(sz)) == 2
+
+    def fon(x=P16, W=P16, M=2, K=32, N=8, y=P16, P=P16, beta=P16, q=P16, s=P16, rs=P16, ws=P16,
+            wsb=1 << 30):
+        return L.bitlinear_forward_online(x, NULL, 1e-5, W, M, K, N, y, 0, P, beta, q, s, rs, ws,
+                                          wsb, NULL)
+
+    assert fon(K=24) == 2
+    assert fon(W=NULL) == 1
+    assert fon(beta=NULL) == 1
+    assert fon(ws=NULL) == 5
+    assert fon(wsb=16) == 5
+    assert fon(W=P17) == 3
+    assert L.bitlinear_forward_online(P16, NULL, 1e-5, P16, 2, 32, 8, P16, 7, P16, P16, P16, P16,
+                                      P16, P16, 1 << 30, NULL) == 4          # bad dtype
+
+    def bwd(gy=P16, q=P16, s=P16, P=P16, beta=P16, M=2, K=32, N=8, gx=P16, gw=P16):
+        return L.bitlinear_backward_ste(gy, q, s, P, beta, M, K, N, gx, gw, NULL)
+
+    assert bwd(M=0) == 0
+    assert bwd(N=6) == 2
+    assert bwd(gx=NULL, gw=NULL) == 1
+    assert bwd(P=NULL) == 1                      # grad_x needs the packed weights
+    assert bwd(q=NULL, gx=NULL) == 1             # grad_w needs the codes
