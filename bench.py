@@ -554,6 +554,48 @@ class DecodeChainWorkload:
             B.bitlinear_act_quant(self.z, L["gs"], eps, q=self.qs, s_x=self.sv[2], rowsum=self.rv[2])
             B.bitlinear_forward_quantized_batch(L["down"], 1)
 
+    def persistent(self, dec):
+        """The same token's steps as one persistent launch (3 steps a layer:
+        q|k|v + o, gate|up, down), on a second pair of residual buffers."""
+        B, WL = self.B, self.WL
+        byname = {(q["layer"], q["name"]): q for q in dec.problems}
+        H, I = WL.HIDDEN, WL.INTERMEDIATE
+        self.pxa = self.x0.reshape(-1).clone()
+        self.pxb = torch.empty_like(self.pxa)
+        self.pz = torch.empty(I, dtype=torch.bfloat16, device="cuda")
+        pqkv = [t.reshape(-1) for t in self.qkv]
+        steps = []
+        for l, L in enumerate(self.layers):
+            steps.append(dict(x=self.pxa, gain=L["ga"], eps=WL.RMS_EPS, problems=[
+                dict(P=byname[(l, n)]["P"], beta=byname[(l, n)]["beta"], y=y)
+                for n, y in zip(("q", "k", "v"), pqkv)] + [
+                dict(P=byname[(l, "o")]["P"], beta=byname[(l, "o")]["beta"], y=self.pxb,
+                     residual=self.pxa)]))
+            steps.append(dict(x=self.pxb, gain=L["gf"], eps=WL.RMS_EPS, problems=[
+                dict(P=L["P2"], beta=L["bg"], beta_up=L["bu"], y=self.pz, kind="gate_up")]))
+            steps.append(dict(x=self.pz, gain=L["gs"], eps=WL.RMS_EPS, problems=[
+                dict(P=byname[(l, "down")]["P"], beta=byname[(l, "down")]["beta"], y=self.pxa,
+                     residual=self.pxb)]))
+        self.chain = B.make_chain(steps)
+        self.chain_ws = B.bitlinear_decode_chain_prepare(self.chain)
+        self.pgraph = capture_graph(self.run_persistent)
+
+    def run_persistent(self):
+        self.pxa.copy_(self.x0.reshape(-1))
+        self.B.bitlinear_decode_chain_run(self.chain_ws, len(self.chain))
+
+    def measure_persistent(self, reps, warmup, world, hbm):
+        ms = timed(self.pgraph.replay, reps, warmup, world) / reps
+        gbs = self.weight_bytes / (ms / 1000.0) / 1e9
+        return {"workload": "dependent decode as one persistent launch: the token's %d steps "
+                            "(per layer q|k|v + o, fused gate|up, down; each step quantises its "
+                            "input in every CTA; grid barrier between steps); attention omitted"
+                            % len(self.chain),
+                "token_us": ms * 1000.0, "tokens_per_s": job_throughput(1, world, ms),
+                "packed_weight_gbs": gbs, "frac_of_hbm": gbs / hbm,
+                "frac_of_nominal_hbm": gbs / NOMINAL_HBM_GBS, "reps": reps,
+                "launches_per_step": 1}
+
     def measure(self, reps, warmup, world, hbm):
         ms = timed(self.graph.replay, reps, warmup, world) / reps
         gbs = self.weight_bytes / (ms / 1000.0) / 1e9
@@ -923,6 +965,8 @@ def main():
         del fw
         dc = DecodeChainWorkload(wl)
         legs["decode_chain"] = dc.measure(reps, rw, world, hbm)
+        dc.persistent(wl)
+        legs["decode_chain_persistent"] = dc.measure_persistent(reps, rw, world, hbm)
         del dc
     if not args.no_prefill:
         pw = PrefillWorkload()

@@ -312,6 +312,62 @@ bl_status bitlinear_backward_ste(const float* grad_y, const int8_t* q, const flo
                                  const uint8_t* P, const float* beta, int64_t M, int64_t K,
                                  int64_t N, float* grad_x, float* grad_w, void* stream);
 
+/* ---- one token through a chain of dependent steps, in one launch -------- */
+
+#define BL_MAX_CHAIN_STEPS 4096
+#define BL_CHAIN_MAX_PROBLEMS 4
+
+typedef enum { BL_CHAIN_BF16 = 0, BL_CHAIN_F32 = 1, BL_CHAIN_GATE_UP = 2 } bl_chain_kind;
+
+/* One projection of a chain step (all pointers device; one token, M = 1). */
+typedef struct {
+    const uint8_t* P;          /* packed weights: [N/4, K], or [N/2, K] for a gate/up pair */
+    void* y;                   /* [N] output: bf16 or fp32 per kind; bf16 z for a pair */
+    const uint16_t* residual;  /* bf16 [N] added after the bf16 rounding, or NULL (bf16 only) */
+    int64_t N;                 /* outputs (I for a gate/up pair from bitlinear_pack_gate_up) */
+    float beta;                /* absmean scale (the gate's for a pair) */
+    float beta_up;             /* the up projection's scale of a pair (else unused) */
+    bl_chain_kind kind;
+} bl_chain_problem;
+
+/* One step: up to BL_CHAIN_MAX_PROBLEMS projections of one input row, each
+ * exactly what bitlinear_forward (M = 1, with its RMSNorm), plus the residual
+ * of bitlinear_forward_quantized or the relu^2 gating of
+ * bitlinear_forward_gate_up, would compute. */
+typedef struct {
+    const uint16_t* x;         /* bf16 [K] input row (16-byte aligned) */
+    const uint16_t* gain;      /* bf16 [K] RMSNorm weight or NULL */
+    float eps;
+    int64_t K;                 /* K % 16 == 0, K <= 8192 */
+    int count;                 /* 1 .. BL_CHAIN_MAX_PROBLEMS */
+    bl_chain_problem p[BL_CHAIN_MAX_PROBLEMS];
+} bl_chain_step;
+
+/* Workspace of a chain of nsteps steps (1 .. BL_MAX_CHAIN_STEPS). */
+bl_status bitlinear_decode_chain_workspace_size(int nsteps, size_t* bytes);
+
+/* Checks the steps and copies their description into the workspace (a
+ * synchronous host-to-device copy; call it once, outside any stream capture).
+ * The buffers the steps name must stay valid while the chain is run. */
+bl_status bitlinear_decode_chain_prepare(const bl_chain_step* steps, int nsteps, void* workspace,
+                                         size_t workspace_bytes);
+
+/* Runs the prepared steps in order, for one token, in one persistent launch
+ * ([BG] "推理侧 BitLinear" for each projection; [MD] model details for the
+ * decoder layer's residual adds and gated relu^2 FFN): step s + 1 sees every
+ * output of step s (a grid-wide barrier separates them), so a step may read
+ * the previous steps' outputs as its input row or residual.  A step's input
+ * row must not be written by that same step (use two residual buffers in
+ * turn: the step that adds o to the residual stream reads x and writes a
+ * second buffer).  Results are bit for bit those of the separate entry points.
+ * Each CTA quantises a step's input itself and the weights of later steps
+ * stream in while it waits at the barrier.  Needs every SM's CTA resident at
+ * once (cooperative launch: BL_ERR_CUDA if the device cannot host it); the
+ * barrier waits are bounded like every other wait (BL_ERR_TIMEOUT through
+ * bitlinear_device_status).  Asynchronous on `stream`. */
+bl_status bitlinear_decode_chain_run(void* workspace, size_t workspace_bytes, int nsteps,
+                                     void* stream);
+
 /* ---- forward without any caller-provided memory besides inputs and outputs -- */
 
 /* Size of the library's fixed device scratch used by bitlinear_forward_noalloc. */

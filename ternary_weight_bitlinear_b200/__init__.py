@@ -10,7 +10,8 @@ from .bitlinear import (BL_MAX_K, BL_OUT_BF16, BL_OUT_F32, BitLinearError, LIB_P
                         bitlinear_forward_quantized_batch, bitlinear_forward_gate_up,
                         bitlinear_pack_gate_up, bitlinear_pack_gate_up_workspace_size,
                         bitlinear_forward_online, bitlinear_forward_online_workspace_size,
-                        bitlinear_backward_ste,
+                        bitlinear_backward_ste, make_chain, bitlinear_decode_chain_prepare,
+                        bitlinear_decode_chain_run, bitlinear_decode_chain_workspace_size,
                         make_batch,
                         make_quantized_batch,
                         bitlinear_forward_workspace_size, bitlinear_pack,

@@ -46,6 +46,9 @@ SIGNATURES = {
     "bitlinear_forward_online": ([_P, _P, _F32, _P, _I64, _I64, _I64, _P, _INT, _P, _P, _P, _P, _P,
                                   _P, _SZ, _P], _INT),
     "bitlinear_backward_ste": ([_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P], _INT),
+    "bitlinear_decode_chain_workspace_size": ([_INT, ctypes.POINTER(_SZ)], _INT),
+    "bitlinear_decode_chain_prepare": ([_P, _INT, _P, _SZ], _INT),
+    "bitlinear_decode_chain_run": ([_P, _SZ, _INT, _P], _INT),
     "bitlinear_forward_noalloc": ([_P, _P, _F32, _P, _F32, _I64, _I64, _I64, _P, _INT, _P], _INT),
     "bitlinear_device_status": ([_P], _INT),
     "bitlinear_selftest_wait_timeout": ([_I64, _P], _INT),
@@ -66,6 +69,22 @@ class QuantizedProblem(ctypes.Structure):
     """bl_quantized_problem: one matmul on already-quantised activations."""
     _fields_ = [("q", _P), ("s_x", _P), ("rowsum", _P), ("P", _P), ("y", _P), ("residual", _P),
                 ("K", _I64), ("N", _I64), ("beta", _F32), ("y_dtype", _INT)]
+
+
+BL_CHAIN_BF16, BL_CHAIN_F32, BL_CHAIN_GATE_UP = 0, 1, 2
+BL_CHAIN_MAX_PROBLEMS = 4
+
+
+class ChainProblem(ctypes.Structure):
+    """bl_chain_problem: one projection of a chain step (M = 1)."""
+    _fields_ = [("P", _P), ("y", _P), ("residual", _P), ("N", _I64), ("beta", _F32),
+                ("beta_up", _F32), ("kind", _INT)]
+
+
+class ChainStep(ctypes.Structure):
+    """bl_chain_step: up to four projections of one input row."""
+    _fields_ = [("x", _P), ("gain", _P), ("eps", _F32), ("K", _I64), ("count", _INT),
+                ("p", ChainProblem * BL_CHAIN_MAX_PROBLEMS)]
 
 
 class BitLinearError(RuntimeError):
@@ -393,6 +412,51 @@ def bitlinear_backward_ste(grad_y, saved, K, grad_x=True, grad_w=True, stream=No
         _ptr(grad_y), _ptr(saved["q"]), _ptr(saved["s_x"]), _ptr(saved["P"]), _ptr(saved["beta"]),
         M, K, N, _ptr(gx), _ptr(gw), _stream(stream)))
     return gx, gw
+
+
+def make_chain(steps):
+    """bl_chain_step array from dicts: x (bf16 [1,K] or [K]), optional gain,
+    eps, problems = [dict(P, y, beta, optional residual, beta_up, kind)]
+    (kind: "bf16", "f32" or "gate_up"; N is taken from y)."""
+    kinds = {"bf16": BL_CHAIN_BF16, "f32": BL_CHAIN_F32, "gate_up": BL_CHAIN_GATE_UP}
+    arr = (ChainStep * len(steps))()
+    for i, st in enumerate(steps):
+        x = st["x"]
+        _need(x, torch.bfloat16, "x")
+        arr[i].x = x.data_ptr()
+        arr[i].gain = _addr(st.get("gain"))
+        arr[i].eps = float(st.get("eps", 1e-5))
+        arr[i].K = x.numel()
+        probs = st["problems"]
+        arr[i].count = len(probs)
+        for j, pr in enumerate(probs):
+            _need(pr["P"], torch.uint8, "P", 2)
+            arr[i].p[j] = ChainProblem(pr["P"].data_ptr(), pr["y"].data_ptr(),
+                                       _addr(pr.get("residual")), pr["y"].numel(),
+                                       float(pr["beta"]), float(pr.get("beta_up", 0.0)),
+                                       kinds[pr.get("kind", "bf16")])
+    return arr
+
+
+def bitlinear_decode_chain_workspace_size(nsteps):
+    n = ctypes.c_size_t()
+    _check("bitlinear_decode_chain_workspace_size",
+           lib().bitlinear_decode_chain_workspace_size(nsteps, ctypes.byref(n)))
+    return n.value
+
+
+def bitlinear_decode_chain_prepare(chain, workspace=None):
+    """Copy a make_chain() array into a (new or given) device workspace; returns it."""
+    ws = _workspace(bitlinear_decode_chain_workspace_size(len(chain)), "cuda") \
+        if workspace is None else workspace
+    _check("bitlinear_decode_chain_prepare", lib().bitlinear_decode_chain_prepare(
+        ctypes.cast(chain, _P), len(chain), _ptr(ws), ws.numel()))
+    return ws
+
+
+def bitlinear_decode_chain_run(workspace, nsteps, stream=None):
+    _check("bitlinear_decode_chain_run", lib().bitlinear_decode_chain_run(
+        _ptr(workspace), workspace.numel(), nsteps, _stream(stream)))
 
 
 def bitlinear_selftest_wait_timeout(limit_ns, stream=None):

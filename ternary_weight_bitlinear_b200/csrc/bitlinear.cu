@@ -13,6 +13,7 @@
 #include <map>
 #include <mutex>
 #include <tuple>
+#include <vector>
 
 #include "common.cuh"
 #include "decode.cuh"
@@ -22,6 +23,7 @@
 #include "quant.cuh"
 #include "skinny.cuh"
 #include "ste.cuh"
+#include "chain.cuh"
 
 namespace {
 
@@ -126,6 +128,30 @@ bl_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
     if (e != cudaSuccess) {
         record_cuda_error(e, "cudaLaunchKernelEx");
+        cudaGetLastError();
+        return BL_ERR_CUDA;
+    }
+    return BL_OK;
+}
+
+// Cooperative launch: every CTA of the grid is resident at once (or the
+// launch fails), which a kernel with a grid-wide barrier needs.
+template <typename... KArgs, typename... Args>
+bl_status launch_coop(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "cudaLaunchKernelEx (cooperative)");
         cudaGetLastError();
         return BL_ERR_CUDA;
     }
@@ -910,6 +936,106 @@ bl_status bitlinear_backward_ste(const float* grad_y, const int8_t* q, const flo
                      grad_y, q, s_x, M, K, N, grad_w)) != BL_OK)
         return st;
     return BL_OK;
+}
+
+bl_status bitlinear_decode_chain_workspace_size(int nsteps, size_t* bytes) {
+    if (!bytes) return BL_ERR_NULL;
+    if (nsteps < 1 || nsteps > BL_MAX_CHAIN_STEPS) return BL_ERR_SHAPE;
+    *bytes = (size_t)(256 + (int64_t)nsteps * (int64_t)sizeof(ChainStep));
+    return BL_OK;
+}
+
+bl_status bitlinear_decode_chain_prepare(const bl_chain_step* steps, int nsteps, void* workspace,
+                                         size_t workspace_bytes) {
+    size_t need = 0;
+    bl_status st = bitlinear_decode_chain_workspace_size(nsteps, &need);
+    if (st != BL_OK) return st;
+    if (!steps) return BL_ERR_NULL;
+    if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGN;
+    std::vector<ChainStep> host((size_t)nsteps);
+    for (int i = 0; i < nsteps; ++i) {
+        const bl_chain_step& in = steps[i];
+        ChainStep& cs = host[(size_t)i];
+        if (in.count < 1 || in.count > BL_CHAIN_MAX_PROBLEMS) return BL_ERR_SHAPE;
+        if (in.K <= 0 || in.K % 16 != 0 || in.K > kChMaxK) return BL_ERR_SHAPE;
+        if (!in.x) return BL_ERR_NULL;
+        if (!aligned16(in.x) || (in.gain && !aligned16(in.gain))) return BL_ERR_ALIGN;
+        cs = ChainStep{};
+        cs.x = in.x;
+        cs.gain = in.gain;
+        cs.eps = in.eps;
+        cs.K = (int)in.K;
+        cs.count = in.count;
+        int64_t total = 0;
+        for (int j = 0; j < in.count; ++j) {
+            const bl_chain_problem& pj = in.p[j];
+            ChainProblem& cp = cs.p[j];
+            if (!pj.P || !pj.y) return BL_ERR_NULL;
+            if (!aligned16(pj.P)) return BL_ERR_ALIGN;
+            if (pj.kind == BL_CHAIN_GATE_UP) {
+                if (pj.N <= 0 || pj.N % 2 != 0 || pj.residual) return BL_ERR_SHAPE;
+                cp.epi = kEpiGateUp;
+                cp.R = pj.N / 2;
+            } else if (pj.kind == BL_CHAIN_BF16 || pj.kind == BL_CHAIN_F32) {
+                if (pj.N <= 0 || pj.N % 4 != 0) return BL_ERR_SHAPE;
+                if (pj.kind == BL_CHAIN_F32 && pj.residual) return BL_ERR_DTYPE;
+                cp.epi = pj.kind == BL_CHAIN_BF16 ? kEpiBF16 : kEpiF32;
+                cp.R = pj.N / 4;
+            } else {
+                return BL_ERR_DTYPE;
+            }
+            cp.P = pj.P;
+            cp.y = pj.y;
+            cp.residual = pj.residual;
+            cp.N = pj.N;
+            cp.beta = pj.beta;
+            cp.beta2 = pj.beta_up;
+            cp.byte0 = total;
+            total += cp.R * in.K;
+        }
+        cs.total = total;
+    }
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    cudaError_t e = cudaMemcpy(static_cast<char*>(workspace) + 256, host.data(),
+                               sizeof(ChainStep) * (size_t)nsteps, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "cudaMemcpy");
+        cudaGetLastError();
+        return BL_ERR_CUDA;
+    }
+    return BL_OK;
+}
+
+bl_status bitlinear_decode_chain_run(void* workspace, size_t workspace_bytes, int nsteps,
+                                     void* stream) {
+    size_t need = 0;
+    bl_status st = bitlinear_decode_chain_workspace_size(nsteps, &need);
+    if (st != BL_OK) return st;
+    if (!workspace || workspace_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGN;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int occ = prepare_kernel(reinterpret_cast<const void*>(chain_decode_kernel), dev, info,
+                                   kChThreads, kChSmemBytes);
+    if (occ < 1) return BL_ERR_CUDA;
+    unsigned int* bar = static_cast<unsigned int*>(workspace);
+    cudaError_t e = cudaMemsetAsync(bar, 0, sizeof(unsigned int), s);
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "cudaMemsetAsync");
+        cudaGetLastError();
+        return BL_ERR_CUDA;
+    }
+    ChainArgs args;
+    args.steps = reinterpret_cast<const ChainStep*>(static_cast<char*>(workspace) + 256);
+    args.nsteps = nsteps;
+    args.bar = bar;
+    return launch_coop(chain_decode_kernel, dim3((unsigned)info.sms), dim3(kChThreads),
+                       (size_t)kChSmemBytes, s, args);
 }
 
 bl_status bitlinear_quantized_batch_workspace_size(int64_t M, size_t* bytes) {

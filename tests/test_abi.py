@@ -242,3 +242,33 @@ def test_online_and_backward_argument_checks(L):
     assert bwd(gx=NULL, gw=NULL) == 1
     assert bwd(P=NULL) == 1                      # grad_x needs the packed weights
     assert bwd(q=NULL, gx=NULL) == 1             # grad_w needs the codes
+
+
+def test_decode_chain_argument_checks(L):
+    sz = ctypes.c_size_t()
+    assert L.bitlinear_decode_chain_workspace_size(0, ctypes.byref(sz)) == 2
+    assert L.bitlinear_decode_chain_workspace_size(90, ctypes.byref(sz)) == 0
+    assert sz.value > 90 * 64
+    steps = (B.bitlinear.ChainStep * 2)()
+    for st in steps:
+        st.x, st.eps, st.K, st.count = 0x10000, 1e-5, 256, 1
+        st.p[0] = B.bitlinear.ChainProblem(0x10000, 0x10000, None, 128, 1.0, 0.0, 0)
+    ws = ctypes.c_void_p(0x10000)
+    big = 1 << 20
+    assert L.bitlinear_decode_chain_prepare(steps, 2, None, big) == 5
+    assert L.bitlinear_decode_chain_prepare(None, 2, ws, big) == 1
+    steps[1].K = 8208                             # beyond the chain's row limit
+    assert L.bitlinear_decode_chain_prepare(steps, 2, ws, big) == 2
+    steps[1].K = 256
+    steps[1].count = 5
+    assert L.bitlinear_decode_chain_prepare(steps, 2, ws, big) == 2
+    steps[1].count = 1
+    steps[1].p[0].kind = 7
+    assert L.bitlinear_decode_chain_prepare(steps, 2, ws, big) == 4
+    steps[1].p[0].kind = 2                        # a gate/up pair needs an even N, no residual
+    steps[1].p[0].N = 7
+    assert L.bitlinear_decode_chain_prepare(steps, 2, ws, big) == 2
+    steps[1].p[0].N = 128
+    steps[1].p[0].P = 0x10001
+    assert L.bitlinear_decode_chain_prepare(steps, 2, ws, big) == 3
+    assert L.bitlinear_decode_chain_run(ws, 16, 2, None) == 5
