@@ -62,6 +62,11 @@ def parse_args():
                     help="skip the M=4096 prefill measurement reported beside the headline")
     ap.add_argument("--no-comparator", action="store_true",
                     help="skip the bf16 dequantised-matmul comparator")
+    ap.add_argument("--passes", type=int, default=0,
+                    help="token passes per headline step (0: enough for %.1f s of device time)"
+                    % HEADLINE_MIN_S)
+    ap.add_argument("--reps", type=int, default=LEG_REPS,
+                    help="timed repeats of every other leg (profiling runs use a few)")
     return ap.parse_args()
 
 
@@ -471,6 +476,36 @@ class FfnChainWorkload:
                 dict(q=self.q2, s_x=self.s2, rowsum=self.r2, P=L["d"]["P"], beta=L["d"]["beta"],
                      y=self.x, residual=self.x)])
         self.graph = capture_graph(self.run)
+
+    def unfused(self, dec):
+        """The same chain with gate and up as two problems of one batched
+        call, then relu2_mul: 5 launches a layer (the control of the fused pass)."""
+        B = self.B
+        byname = {(q["layer"], q["name"]): q for q in dec.problems}
+        M, I = self.M, self.WL.INTERMEDIATE
+        self.a = torch.empty((M, I), dtype=torch.bfloat16, device="cuda")
+        self.b = torch.empty((M, I), dtype=torch.bfloat16, device="cuda")
+        for l, L in enumerate(self.layers):
+            g, u = byname[(l, "gate")], byname[(l, "up")]
+            L["gu"] = B.make_quantized_batch([
+                dict(q=self.q1, s_x=self.s1, rowsum=self.r1, P=g["P"], beta=g["beta"], y=self.a),
+                dict(q=self.q1, s_x=self.s1, rowsum=self.r1, P=u["P"], beta=u["beta"], y=self.b)])
+        self.graph_unfused = capture_graph(self.run_unfused)
+
+    def run_unfused(self):
+        B, eps, M = self.B, self.WL.RMS_EPS, self.M
+        self.x.copy_(self.x0)
+        for L in self.layers:
+            B.bitlinear_act_quant(self.x, L["gi"], eps, q=self.q1, s_x=self.s1, rowsum=self.r1)
+            B.bitlinear_forward_quantized_batch(L["gu"], M, workspace=self.ws)
+            B.bitlinear_relu2_mul(self.a, self.b, out=self.z)
+            B.bitlinear_act_quant(self.z, L["gs"], eps, q=self.q2, s_x=self.s2, rowsum=self.r2)
+            B.bitlinear_forward_quantized_batch(L["dn"], M, workspace=self.ws)
+
+    def measure_unfused(self, reps, warmup, world):
+        ms = timed(self.graph_unfused.replay, reps, warmup, world) / reps
+        return {"chain_us": ms * 1000.0, "tokens_per_s": job_throughput(self.M, world, ms),
+                "launches_per_step": 5 * len(self.layers), "reps": reps}
 
     def run(self):
         B, eps, M = self.B, self.WL.RMS_EPS, self.M
@@ -916,9 +951,12 @@ def main():
     # in one batched forward call (one quantise launch + one GEMV launch).  A
     # step is `passes` back-to-back passes of that call, enough that the K
     # timed steps cover at least HEADLINE_MIN_S of device time.
-    probe_ms = timed(head.replay, 20, max(args.warmup, 3), world) / 20
-    passes = int(max(1, min(2000, np.ceil(HEADLINE_MIN_S * 1000.0 / (args.steps * probe_ms)))))
-    passes = int(max_over_ranks(passes, world))
+    if args.passes > 0:
+        passes = args.passes
+    else:
+        probe_ms = timed(head.replay, 20, max(args.warmup, 3), world) / 20
+        passes = int(max(1, min(2000, np.ceil(HEADLINE_MIN_S * 1000.0 / (args.steps * probe_ms)))))
+        passes = int(max_over_ranks(passes, world))
 
     def head_step():
         for _ in range(passes):
@@ -930,7 +968,7 @@ def main():
     ms_step = ms / args.steps
     value = job_throughput(wl.M * passes * args.steps, world, ms)
 
-    reps, rw = LEG_REPS, max(args.warmup, 3)
+    reps, rw = args.reps, max(args.warmup, 3)
     # the GEMV kernel alone on the same batch (pre-quantised codes): its roofline
     ms_gemv = max_over_ranks(timed(wl.graphs["gemv_token"].replay, reps, rw, world), world)
     variants = {}
@@ -962,6 +1000,8 @@ def main():
         legs["skinny"] = skinny
         fw = FfnChainWorkload(wl)
         legs["ffn_chain"] = fw.measure(reps, rw, world, hbm)
+        fw.unfused(wl)
+        legs["ffn_chain"]["unfused_gate_up"] = fw.measure_unfused(reps, rw, world)
         del fw
         dc = DecodeChainWorkload(wl)
         legs["decode_chain"] = dc.measure(reps, rw, world, hbm)

@@ -453,11 +453,13 @@ unsigned long long next_epoch() {
 // boundaries.
 bl_status run_skinny(const DecodeJob* jobs, int count, int64_t M, void* ws, size_t ws_bytes, int dev,
                      const DeviceInfo& info, cudaStream_t stream) {
-    if (prepare_kernel(reinterpret_cast<const void*>(skinny_tc_kernel), dev, info, kSkThreads,
-                       kSkSmemBytes) < 0)
-        return BL_ERR_CUDA;
-    static thread_local SkBatch b;  // ~22 KB: kept off the stack
     const int npad = (int)sk_npad(M);
+    const bool ew4 = sk_epi_warps(npad) == 4;
+    const int threads = sk_threads(sk_epi_warps(npad));
+    const void* kfn = ew4 ? reinterpret_cast<const void*>(skinny_tc_kernel<4>)
+                          : reinterpret_cast<const void*>(skinny_tc_kernel<8>);
+    if (prepare_kernel(kfn, dev, info, threads, kSkSmemBytes) < 0) return BL_ERR_CUDA;
+    static thread_local SkBatch b;  // ~22 KB: kept off the stack
     const bool split = ws && ws_bytes >= (size_t)sk_ws_bytes(M);
     for (int c0 = 0; c0 < count; c0 += kSkCap) {
         const int n = std::min(kSkCap, count - c0);
@@ -499,8 +501,10 @@ bl_status run_skinny(const DecodeJob* jobs, int count, int64_t M, void* ws, size
         b.epoch = next_epoch();
         const int64_t grid = std::max<int64_t>(
             1, std::min<int64_t>(items, std::min<int64_t>(info.sms, kSkMaxGrid)));
-        bl_status st = launch(skinny_tc_kernel, dim3((unsigned)grid), dim3(kSkThreads),
-                              (size_t)kSkSmemBytes, stream, b);
+        bl_status st = ew4 ? launch(skinny_tc_kernel<4>, dim3((unsigned)grid), dim3((unsigned)threads),
+                                    (size_t)kSkSmemBytes, stream, b)
+                           : launch(skinny_tc_kernel<8>, dim3((unsigned)grid), dim3((unsigned)threads),
+                                    (size_t)kSkSmemBytes, stream, b);
         if (st != BL_OK) return st;
     }
     return BL_OK;

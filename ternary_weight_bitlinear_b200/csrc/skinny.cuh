@@ -34,10 +34,12 @@
 //  * One thread issues tcgen05.mma.cta_group::1.kind::i8 with A (weights) from
 //    TMEM and B (tokens, N = M rounded up to 16) from shared memory into one
 //    of two TMEM accumulators, and releases the ring slots with
-//    tcgen05.commit.
-//  * Eight epilogue warps (two per TMEM lane quadrant, each half of the
-//    tokens) take a finished row tile: tcgen05.ld, minus the row sums,
-//    rescale (exact division through the token's reciprocal), store.
+//    tcgen05.commit (one commit per item frees its ring stage and its TMEM
+//    slot).
+//  * Four epilogue warps (one per TMEM lane quadrant) up to 16 tokens, eight
+//    (two per quadrant, each half of the tokens) beyond, take a finished row
+//    tile: tcgen05.ld, minus the row sums, rescale (exact division through
+//    the token's reciprocal), store.
 //  * A row tile whose items straddle several CTAs is finished by whichever of
 //    them gets there last: each leaves its int32 partial sums in the caller's
 //    workspace and counts itself in on the tile's counter (an atomic
@@ -72,9 +74,13 @@ constexpr int kSkTeams = 2;                          // expansion teams (4 warps
 constexpr int kSkMmaWarp = 1;
 constexpr int kSkExpWarp0 = 2;
 constexpr int kSkEpiWarp0 = kSkExpWarp0 + 4 * kSkTeams;
-constexpr int kSkEpiWarps = 8;                       // two per lane quadrant, each half the tokens
-constexpr int kSkEpiThreads = 32 * kSkEpiWarps;
-constexpr int kSkThreads = 32 * (kSkEpiWarp0 + kSkEpiWarps);
+// epilogue warps: 4 (one per lane quadrant, all tokens) up to 16 tokens, 8
+// (two per lane quadrant, each half the tokens) beyond; the register budget
+// of the 4-warp form is 128 per thread, of the 8-warp form 96 (below).  On
+// this GPU the 4-warp form is ~3 % faster at 8 and 16 tokens and ~12 %
+// slower at 32, where the epilogue's share of an item grows.
+__host__ __device__ constexpr int sk_threads(int ew) { return 32 * (kSkEpiWarp0 + ew); }
+__host__ __device__ constexpr int sk_epi_warps(int npad) { return npad <= 16 ? 4 : 8; }
 constexpr int kSkCap = 64;                           // problems per launch
 constexpr int kSkMaxGrid = 160;                      // CTAs per launch (>= SM count)
 // TMEM columns: A ring [0, 384); accumulators [384, 512): two buffers of 64
@@ -82,7 +88,7 @@ constexpr uint32_t kSkTmemCols = 512;
 constexpr uint32_t kSkACols = 32 * kSkKB;            // 128 columns (512 K bytes) per slot
 constexpr uint32_t kSkDCol0 = kSkACols * kSkASlots;
 constexpr uint32_t kSkDBuf = 64;
-constexpr int kSkNumBars = 2 * kSkMaxStages + 2 * kSkASlots + 2 * 2 + 1;
+constexpr int kSkNumBars = 2 * kSkMaxStages + kSkASlots + 2 * 2 + 1;
 constexpr int kSkOffBar = kSkRingBytes;
 // tmem address | last-arriver flag | per-problem token constants (s_x,
 // RN(1/s_x), row sums) for the epilogue
@@ -92,10 +98,15 @@ constexpr int kSkSmemBytes = kSkOffTok + 12 * kSkMaxTokens + 1024;
 static_assert(kSkSmemBytes <= 227 * 1024, "shared memory budget");
 static_assert(kSkPBytes % 1024 == 0, "swizzle atoms stay 1024-aligned");
 static_assert(kSkMaxStages * (kSkPBytes + kSkKB * 16 * kSkBK) <= kSkRingBytes, "ring holds 8 stages at npad 16");
+// the ring's "item done" barriers also free the TMEM slots: an expansion team
+// waits on item g - kSkASlots, which needs a ring of more than kSkASlots stages
+static_assert(kSkRingBytes / (kSkPBytes + kSkKB * kSkMaxTokens * kSkBK) > kSkASlots, "ring depth");
 static_assert(kSkDCol0 + 2 * kSkDBuf <= kSkTmemCols && kSkMaxTokens <= (int)kSkDBuf, "TMEM budget");
 // each of the four schedulers of an SM holds 16384 registers: with 18 warps one
-// scheduler holds 5, so at most 96 registers a thread (launch bounds below)
-static_assert((kSkThreads / 32 + 3) / 4 * 32 * 96 <= 16384, "register budget of one CTA per SM");
+// scheduler holds 5, so at most 96 registers a thread; with 14, 4 and 128
+// (launch bounds below)
+static_assert((sk_threads(8) / 32 + 3) / 4 * 32 * 96 <= 16384, "register budget, 8 epilogue warps");
+static_assert((sk_threads(4) / 32 + 3) / 4 * 32 * 128 <= 16384, "register budget, 4 epilogue warps");
 
 struct SkProblem {
     const float* s_x;          // [M]
@@ -241,13 +252,15 @@ __device__ __forceinline__ uint32_t sk_idesc(int npad) {
     return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(npad >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-// Named barrier among the eight epilogue warps.
+// Named barrier among the EW epilogue warps.
+template <int EW>
 __device__ __forceinline__ void sk_epi_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kSkEpiThreads) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * EW) : "memory");
 }
 
 // The same barrier, returning whether `pred` held in all of them (so that they
 // always take the same exits and never leave one another waiting).
+template <int EW>
 __device__ __forceinline__ bool sk_epi_all(bool pred) {
     uint32_t r;
     asm volatile(
@@ -256,7 +269,7 @@ __device__ __forceinline__ bool sk_epi_all(bool pred) {
         "bar.red.and.pred b, 1, %2, a;\n\t"
         "selp.u32 %0, 1, 0, b;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)pred), "n"(kSkEpiThreads)
+        : "r"((uint32_t)pred), "n"(32 * EW)
         : "memory");
     return r != 0;
 }
@@ -323,19 +336,21 @@ __device__ __forceinline__ void sk_store_gate_up(const SkProblem& pr, int m, int
     static_cast<uint16_t*>(pr.y)[(int64_t)m * pr.N + n] = relu2_mul_one(a, bb);
 }
 
-__global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_constant__ SkBatch b) {
+template <int EW>
+__global__ void __launch_bounds__(sk_threads(EW), 1) skinny_tc_kernel(const __grid_constant__ SkBatch b) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* sm = smem_raw + (base - raw);
     const uint32_t bars = base + kSkOffBar;
     auto full_bar = [&](int s) { return bars + 8u * s; };
+    // empty_bar(s): the MMAs of the item in ring stage s are done, which frees
+    // the stage and the item's TMEM slot (one commit per item)
     auto empty_bar = [&](int s) { return bars + 8u * (kSkMaxStages + s); };
     auto afull_bar = [&](int a) { return bars + 8u * (2 * kSkMaxStages + a); };
-    auto aempty_bar = [&](int a) { return bars + 8u * (2 * kSkMaxStages + kSkASlots + a); };
-    auto dfull_bar = [&](int d) { return bars + 8u * (2 * kSkMaxStages + 2 * kSkASlots + d); };
-    auto dempty_bar = [&](int d) { return bars + 8u * (2 * kSkMaxStages + 2 * kSkASlots + 2 + d); };
-    const uint32_t mma_done_bar = bars + 8u * (2 * kSkMaxStages + 2 * kSkASlots + 4);
+    auto dfull_bar = [&](int d) { return bars + 8u * (2 * kSkMaxStages + kSkASlots + d); };
+    auto dempty_bar = [&](int d) { return bars + 8u * (2 * kSkMaxStages + kSkASlots + 2 + d); };
+    const uint32_t mma_done_bar = bars + 8u * (2 * kSkMaxStages + kSkASlots + 4);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSkOffTmem);
     volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(sm + kSkOffTmem + 4);
     // ring stage: 4 packed boxes (4 KB each) | 4 token boxes (npad x 128 each)
@@ -351,13 +366,10 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        for (int a = 0; a < kSkASlots; ++a) {
-            mbar_init(afull_bar(a), 4);
-            mbar_init(aempty_bar(a), 1);
-        }
+        for (int a = 0; a < kSkASlots; ++a) mbar_init(afull_bar(a), 4);
         for (int d = 0; d < 2; ++d) {
             mbar_init(dfull_bar(d), 1);
-            mbar_init(dempty_bar(d), kSkEpiWarps);
+            mbar_init(dempty_bar(d), EW);
         }
         mbar_init(mma_done_bar, 1);
         mbar_init_fence();
@@ -455,7 +467,6 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
                     acol += 8u;
                 }
                 tc_commit(empty_bar(s));
-                tc_commit(aempty_bar(a));
                 const bool last = g + 1 == n_items || cur.ks + 1 == cur.kst;
                 first = last;
                 if (last) {
@@ -484,8 +495,11 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
         }
         for (uint32_t g = (uint32_t)team; g < n_items && ok; g += kSkTeams) {
             const int s = (int)(g % (uint32_t)nstages), a = (int)(g % kSkASlots);
+            // TMEM slot a is free once item g - kSkASlots (which used it) is done
+            const uint32_t gp = g - kSkASlots;
             const bool got = mbar_wait(full_bar(s), (g / nstages) & 1u) &&
-                             mbar_wait(aempty_bar(a), ((g / kSkASlots) & 1u) ^ 1u);
+                             (g < (uint32_t)kSkASlots ||
+                              mbar_wait(empty_bar((int)(gp % (uint32_t)nstages)), (gp / nstages) & 1u));
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
             const int nkb = (cur.valid_k() + kSkBK - 1) / kSkBK;
@@ -514,15 +528,16 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
         pdl_launch_dependents();
         // ---------------- epilogue: one weight row, half of the tokens per thread ----------------
         const int ew = warp - kSkEpiWarp0;
-        const int qd = warp & 3, half = ew >> 2;
+        const int qd = warp & 3, half = EW == 8 ? ew >> 2 : 0;
         const int bit = lane >> 3, j = lane & 7;
         const int row128 = 32 * qd + lane;  // D row (TMEM lane)
         float* tok_s = reinterpret_cast<float*>(sm + kSkOffTok);
         float* tok_y = tok_s + kSkMaxTokens;
         int* tok_rs = reinterpret_cast<int*>(tok_y + kSkMaxTokens);
-        const int et = threadIdx.x - 32 * kSkEpiWarp0;  // 0..255
-        // this thread's token columns [c0, c1): halves of npad in 16-column steps
-        const int hc = ((b.npad / 2) + 15) & ~15;
+        const int et = threadIdx.x - 32 * kSkEpiWarp0;  // 0..32 EW - 1
+        // this thread's token columns [c0, c1): all of them (4 warps, npad =
+        // 16), or halves of npad in 16-column steps (8 warps)
+        const int hc = EW == 8 ? ((b.npad / 2) + 15) & ~15 : b.npad;
         const int c0 = half * hc, c1 = min(b.npad, c0 + hc);
         const uint32_t ep32 = (uint32_t)b.epoch;
         int staged = -1;
@@ -536,14 +551,14 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
             SkProblem pr = b.p[cur.p];
             if (pr.beta_dev) pr.beta = __ldcg(pr.beta_dev);
             if (staged != cur.p) {  // this problem's token scales and row sums, once
-                sk_epi_sync();
+                sk_epi_sync<EW>();
                 if (et < b.M) {
                     const float sx = pr.epi == kEpiI32 ? 1.0f : __ldcg(pr.s_x + et);
                     tok_s[et] = sx;
                     tok_y[et] = __frcp_rn(sx);
                     tok_rs[et] = __ldcg(pr.rowsum + et);
                 }
-                sk_epi_sync();
+                sk_epi_sync<EW>();
                 staged = cur.p;
             }
             const int64_t tile_first = pr.item0 + (int64_t)cur.tile * pr.kst;
@@ -552,7 +567,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
             const bool split = item > tile_first || part_end < tile_end;
             const int d = (int)(tl & 1);
             const bool got = mbar_wait(dfull_bar(d), (tl >> 1) & 1u);
-            if (!sk_epi_all(got)) { ok = false; break; }
+            if (!sk_epi_all<EW>(got)) { ok = false; break; }
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(32 * qd) << 16) + kSkDCol0 + (uint32_t)d * kSkDBuf;
             bool write = true;
@@ -573,13 +588,13 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_tc_kernel(const __grid_c
                     if (c0 + k < c1)
                         *reinterpret_cast<uint4*>(mine + c0 + k) = make_uint4(v[k], v[k + 1], v[k + 2], v[k + 3]);
                 __threadfence();
-                sk_epi_sync();
+                sk_epi_sync<EW>();
                 if (et == 0) {
                     bool aok = true;
                     *last_flag = sk_arrive_last(b.ctr + cf, ep32, (uint32_t)(cl - cf + 1), aok) ? 1u : 0u;
                     if (!aok) *last_flag = 2u;
                 }
-                sk_epi_sync();
+                sk_epi_sync<EW>();
                 const uint32_t lf = *last_flag;
                 if (lf == 2u) ok = false;
                 write = lf == 1u;
