@@ -23,6 +23,8 @@ residual_add      bf16(x + d)
 ffn_block         one FFN block of the 30-layer chain
 online_forward    weight scale + ternarise on this call, then forward (online QAT)
 ste_backward      linear backward on the dequantised operands (straight-through)
+rope, attn_decode the attention block's RoPE and GQA decode attention, float64
+                  numpy (``oracle/attention.py``)
 """
 import ctypes
 import os
@@ -30,6 +32,7 @@ import os
 import numpy as np
 
 from . import build as _build
+from .attention import attn_decode, rope, rope_inv_freq  # noqa: F401
 
 _LIB = None
 _PARALLEL = False
