@@ -25,6 +25,7 @@ import ctypes
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -686,6 +687,48 @@ class Bf16Comparator:
                 "reps": reps}
 
 
+class AttentionWorkload:
+    """The attention block of one decode token at the 2B4T head shapes (20
+    query heads, 5 key/value heads of 128): RoPE of its q and k rows, then the
+    grouped-query attention over an L-position key/value cache (the model's
+    2048 positions at most), both through the public entry points, captured
+    in a CUDA graph of `calls` token-layers.  Bytes per call: the L cached key
+    and value rows read once (L * 640 * 2 * 2) plus q, k and the output."""
+
+    def __init__(self, L, calls=30):
+        import ternary_weight_bitlinear_b200 as B
+        from ternary_weight_bitlinear_b200 import workloads as WL
+        self.B, self.L, self.calls = B, L, calls
+        H, Hkv, d = WL.Q_HEADS, WL.KV_HEADS, WL.HEAD_DIM
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+        q, k, v = WL.attention_decode_inputs(L, seed=L + 3)
+        self.q, self.k, self.v = dev(q), dev(k), dev(v)
+        self.knew = self.k[L - 1].reshape(1, Hkv * d)  # the token's own key row, rotated in place
+        self.qm = self.q.reshape(1, H * d)
+        self.pos = torch.full((1,), L - 1, dtype=torch.int32, device="cuda")
+        self.out = torch.empty(H * d, dtype=torch.bfloat16, device="cuda")
+        self.ws = torch.empty(max(16, B.bitlinear_attn_decode_workspace_size(L, H, Hkv, d)),
+                              dtype=torch.uint8, device="cuda")
+        self.scale = 1.0 / math.sqrt(d)
+        self.H, self.Hkv = H, Hkv
+        self.bytes = L * Hkv * d * 2 * 2 + 2 * H * d * 2 + Hkv * d * 2 * 2
+        self.graph = capture_graph(self.run)
+
+    def run(self):
+        B = self.B
+        for _ in range(self.calls):
+            B.bitlinear_rope(self.qm, self.pos, self.H, 500000.0, out=self.qm)
+            B.bitlinear_rope(self.knew, self.pos, self.Hkv, 500000.0, out=self.knew)
+            B.bitlinear_attn_decode(self.q, self.k, self.v, self.L, self.H, self.Hkv, self.scale,
+                                    out=self.out, workspace=self.ws)
+
+    def measure(self, reps, warmup, world, hbm):
+        ms = timed(self.graph.replay, reps, warmup, world) / reps / self.calls
+        gbs = self.bytes / (ms / 1000.0) / 1e9
+        return {"L": self.L, "layer_us": ms * 1000.0, "gbs": gbs, "frac_of_hbm": gbs / hbm,
+                "launches_per_layer": 4, "reps": reps}
+
+
 def capture_graph(fn):
     """Run fn once on a side stream (caches, attributes), then capture it."""
     s = torch.cuda.Stream()
@@ -1008,6 +1051,15 @@ def main():
         dc.persistent(wl)
         legs["decode_chain_persistent"] = dc.measure_persistent(reps, rw, world, hbm)
         del dc
+    if not args.no_skinny:
+        att = {"workload": "attention block of one decode token, 2B4T heads (20 query, 5 key/value "
+                           "of 128): RoPE of q and of the new k row, grouped-query attention over "
+                           "an L-position cache; 30 token-layers per graph", "by_L": {}}
+        for Ls in (512, 2048):
+            aw = AttentionWorkload(Ls)
+            att["by_L"][str(Ls)] = aw.measure(reps, rw, world, hbm)
+            del aw
+        legs["attention_decode"] = att
     if not args.no_prefill:
         pw = PrefillWorkload()
         legs["prefill"] = pw.measure(reps, rw, world)

@@ -407,6 +407,53 @@ bl_status bitlinear_forward_noalloc(const uint16_t* x, const uint16_t* gain, flo
 bl_status bitlinear_relu2_mul(const uint16_t* a, const uint16_t* b, int64_t n, uint16_t* z,
                               void* stream);
 
+/* ---- attention block of the decoder layer (RoPE, GQA decode attention) ---- */
+
+/* Rotary position embeddings ([MD] model details: the decoder uses RoPE;
+ * BitNetConfig: 20 heads of 128 dimensions for q, 5 for k, 2048 positions).
+ * The pages give no formula; the rotate-half form is used: for every head and
+ * i < head_dim/2 the pair (x[i], x[i + head_dim/2]) is turned by the angle
+ * a = pos[m] * theta^(-2i/head_dim):
+ *   y[i]              = x[i] cos a - x[i + head_dim/2] sin a,
+ *   y[i + head_dim/2] = x[i + head_dim/2] cos a + x[i] sin a,
+ * each evaluated in binary64 and rounded once to bf16.
+ *   x, y      device bf16 [M, heads * head_dim] (y may equal x: in place).
+ *   pos       device int32 [M] token positions.
+ *   theta     base of the frequencies (> 0, finite; rope_theta).
+ * head_dim even and <= 1024; heads, M <= 65535. */
+bl_status bitlinear_rope(const uint16_t* x, const int32_t* pos, int64_t M, int64_t heads,
+                         int64_t head_dim, float theta, uint16_t* y, void* stream);
+
+/* Workspace bitlinear_attn_decode needs for this shape (depends on the
+ * current device's SM count). */
+bl_status bitlinear_attn_decode_workspace_size(int64_t L, int64_t q_heads, int64_t kv_heads,
+                                               int64_t head_dim, size_t* bytes);
+
+/* Grouped-query attention of one decode token over its key/value cache ([MD]
+ * BitNetConfig: num_attention_heads 20, num_key_value_heads 5 -- each
+ * key/value head serves a group of query heads; model details: the layer
+ * order q, k, v -> RoPE + attention -> attn_sub_norm -> o).  The pages give
+ * no formula; the textbook one is used: query head h reads key/value head
+ * g = h / (q_heads / kv_heads) and
+ *   out[h] = sum_j p_j v[j, g],  p = softmax_j((q[h] . k[j, g]) * scale),
+ * over the L cached positions (the current token's key and value included).
+ * Arithmetic in binary32 (exp2 of log2-scaled scores, split over the cache
+ * and merged), output rounded to bf16; it matches the exact value within a
+ * stated tolerance, not bit for bit.
+ *   q         device bf16 [q_heads * head_dim] (after RoPE).
+ *   k_cache   device bf16 [>= L, kv_heads, head_dim], 16-byte aligned
+ *             (positions past L are not read).
+ *   v_cache   device bf16 [>= L, kv_heads, head_dim], 16-byte aligned.
+ *   scale     score multiplier (1/sqrt(head_dim) in the model).
+ *   out       device bf16 [q_heads * head_dim].
+ *   workspace device, 16-byte aligned, at least
+ *             bitlinear_attn_decode_workspace_size bytes.
+ * head_dim 64 or 128; q_heads / kv_heads in {1, 2, 4, 8}; L >= 1. */
+bl_status bitlinear_attn_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                                int64_t L, int64_t q_heads, int64_t kv_heads, int64_t head_dim,
+                                float scale, uint16_t* out, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
 /* ---- device status -------------------------------------------------------- */
 
 /* Synchronises `stream`, then returns and clears the library's device status

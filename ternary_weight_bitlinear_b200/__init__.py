@@ -18,4 +18,5 @@ from .bitlinear import (BL_MAX_K, BL_OUT_BF16, BL_OUT_F32, BitLinearError, LIB_P
                         bitlinear_pack_ternary, bitlinear_pack_workspace_size,
                         bitlinear_quantized_batch_workspace_size,
                         bitlinear_selftest_wait_timeout,
-                        bitlinear_relu2_mul, bitlinear_unpack, lib, status_string)
+                        bitlinear_relu2_mul, bitlinear_unpack, lib, status_string,
+                        bitlinear_rope, bitlinear_attn_decode, bitlinear_attn_decode_workspace_size)

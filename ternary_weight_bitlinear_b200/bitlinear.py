@@ -38,6 +38,9 @@ SIGNATURES = {
                                     _INT),
     "bitlinear_accumulate": ([_P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "bitlinear_relu2_mul": ([_P, _P, _I64, _P, _P], _INT),
+    "bitlinear_rope": ([_P, _P, _I64, _I64, _I64, _F32, _P, _P], _INT),
+    "bitlinear_attn_decode_workspace_size": ([_I64, _I64, _I64, _I64, ctypes.POINTER(_SZ)], _INT),
+    "bitlinear_attn_decode": ([_P, _P, _P, _I64, _I64, _I64, _I64, _F32, _P, _P, _SZ, _P], _INT),
     "bitlinear_pack_gate_up_workspace_size": ([_I64, _I64, ctypes.POINTER(_SZ)], _INT),
     "bitlinear_pack_gate_up": ([_P, _P, _I64, _I64, _P, _P, _P, _SZ, _P], _INT),
     "bitlinear_forward_gate_up": ([_P, _P, _P, _P, _F32, _F32, _I64, _I64, _I64, _P, _P, _SZ, _P],
@@ -329,6 +332,44 @@ def bitlinear_relu2_mul(a, b, out=None, stream=None):
     _check("bitlinear_relu2_mul", lib().bitlinear_relu2_mul(_ptr(a), _ptr(b), a.numel(), _ptr(z),
                                                             _stream(stream)))
     return z
+
+
+def bitlinear_rope(x, pos, heads, theta, out=None, stream=None):
+    """RoPE of bf16 x [M, heads * head_dim] at int32 positions pos [M] (out may be x)."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(pos, torch.int32, "pos", 1)
+    M, W = x.shape
+    if W % heads:
+        raise TypeError("x's width must be heads * head_dim")
+    y = torch.empty_like(x) if out is None else out
+    _check("bitlinear_rope", lib().bitlinear_rope(_ptr(x), _ptr(pos), M, heads, W // heads, float(theta),
+                                                  _ptr(y), _stream(stream)))
+    return y
+
+
+def bitlinear_attn_decode_workspace_size(L, q_heads, kv_heads, head_dim):
+    n = ctypes.c_size_t()
+    _check("bitlinear_attn_decode_workspace_size",
+           lib().bitlinear_attn_decode_workspace_size(L, q_heads, kv_heads, head_dim, ctypes.byref(n)))
+    return n.value
+
+
+def bitlinear_attn_decode(q, k_cache, v_cache, L, q_heads, kv_heads, scale, out=None, workspace=None,
+                          stream=None):
+    """One decode token's GQA attention: q bf16 [q_heads * d], caches bf16
+    [>= L, kv_heads, d] -> bf16 [q_heads * d]."""
+    _need(q, torch.bfloat16, "q")
+    _need(k_cache, torch.bfloat16, "k_cache")
+    _need(v_cache, torch.bfloat16, "v_cache")
+    d = q.numel() // q_heads
+    y = torch.empty(q_heads * d, dtype=torch.bfloat16, device=q.device) if out is None else out
+    nbytes = bitlinear_attn_decode_workspace_size(L, q_heads, kv_heads, d)
+    ws = _workspace(nbytes, q.device) if workspace is None else workspace
+    _check("bitlinear_attn_decode",
+           lib().bitlinear_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), L, q_heads, kv_heads, d,
+                                       float(scale), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
+                                       _stream(stream)))
+    return y
 
 
 def bitlinear_pack_gate_up_workspace_size(I, K):

@@ -9,6 +9,7 @@
 #include <atomic>
 #include <chrono>
 #include <climits>
+#include <cmath>
 #include <cstdio>
 #include <map>
 #include <mutex>
@@ -24,6 +25,7 @@
 #include "skinny.cuh"
 #include "ste.cuh"
 #include "chain.cuh"
+#include "attn.cuh"
 
 namespace {
 
@@ -748,6 +750,46 @@ bl_status forward_impl(const uint16_t* x, const uint16_t* gain, float eps, const
 
 }  // namespace
 
+namespace {
+
+// Positions per split: enough splits for two CTAs per SM over the key/value
+// heads, at least 32 positions (one warp's block) each.
+int64_t attn_chunk(int64_t L, int64_t kv_heads, int sms) {
+    const int64_t target = std::max<int64_t>(1, (2 * (int64_t)sms + kv_heads - 1) / kv_heads);
+    const int64_t per = (L + target - 1) / target;
+    return std::max<int64_t>(32, (per + 31) / 32 * 32);
+}
+
+bl_status attn_check(int64_t L, int64_t q_heads, int64_t kv_heads, int64_t head_dim) {
+    if (L <= 0 || L > INT32_MAX || kv_heads <= 0 || q_heads <= 0 || q_heads % kv_heads != 0)
+        return BL_ERR_SHAPE;
+    const int64_t group = q_heads / kv_heads;
+    if (group != 1 && group != 2 && group != 4 && group != 8) return BL_ERR_SHAPE;
+    if (head_dim != 64 && head_dim != 128) return BL_ERR_SHAPE;
+    if (kv_heads > 65535 || q_heads > 65535) return BL_ERR_SHAPE;
+    // splits <= L / 32 must fit the merge kernel's table
+    if ((L + 31) / 32 > kAttnMaxSplits) return BL_ERR_SHAPE;
+    return BL_OK;
+}
+
+template <int D>
+bl_status attn_launch_d(const AttnArgs& a, int group, int64_t splits, int64_t q_heads, uint16_t* out,
+                        cudaStream_t stream) {
+    const dim3 grid((unsigned)splits, (unsigned)a.kv_heads);
+    bl_status st;
+    switch (group) {
+        case 1: st = launch(attn_split_kernel<D, 1>, grid, dim3(kAttnThreads), 0, stream, a); break;
+        case 2: st = launch(attn_split_kernel<D, 2>, grid, dim3(kAttnThreads), 0, stream, a); break;
+        case 4: st = launch(attn_split_kernel<D, 4>, grid, dim3(kAttnThreads), 0, stream, a); break;
+        default: st = launch(attn_split_kernel<D, 8>, grid, dim3(kAttnThreads), 0, stream, a); break;
+    }
+    if (st != BL_OK) return st;
+    return launch(attn_combine_kernel<D>, dim3((unsigned)q_heads), dim3(D), 0, stream,
+                  (const float*)a.part, (int)splits, (int)q_heads, out);
+}
+
+}  // namespace
+
 extern "C" {
 
 bl_status bitlinear_forward(const uint16_t* x, const uint16_t* gain, float eps, const uint8_t* P,
@@ -1115,6 +1157,71 @@ bl_status bitlinear_relu2_mul(const uint16_t* a, const uint16_t* b, int64_t n, u
     const int64_t threads = (n + 7) / 8;
     return launch(relu2_mul_kernel, dim3((unsigned)((threads + kGlueThreads - 1) / kGlueThreads)),
                   dim3(kGlueThreads), 0, static_cast<cudaStream_t>(stream), a, b, n, z);
+}
+
+// ---- attention block: RoPE and grouped-query decode attention ----------------
+
+bl_status bitlinear_rope(const uint16_t* x, const int32_t* pos, int64_t M, int64_t heads,
+                         int64_t head_dim, float theta, uint16_t* y, void* stream) {
+    if (M < 0 || heads <= 0 || head_dim <= 0 || head_dim % 2 != 0 || head_dim > 1024 ||
+        heads > 65535 || M > 65535)
+        return BL_ERR_SHAPE;
+    if (!(theta > 0.0f) || !std::isfinite(theta)) return BL_ERR_SHAPE;
+    if (M == 0) return BL_OK;
+    if (!x || !pos || !y) return BL_ERR_NULL;
+    int dev;
+    DeviceInfo info;
+    bl_status st;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    return launch(rope_kernel, dim3((unsigned)heads, (unsigned)M), dim3((unsigned)(head_dim / 2)), 0,
+                  static_cast<cudaStream_t>(stream), x, pos, (int)heads, (int)head_dim,
+                  std::log((double)theta), y);
+}
+
+
+bl_status bitlinear_attn_decode_workspace_size(int64_t L, int64_t q_heads, int64_t kv_heads,
+                                               int64_t head_dim, size_t* bytes) {
+    if (!bytes) return BL_ERR_NULL;
+    bl_status st;
+    if ((st = attn_check(L, q_heads, kv_heads, head_dim)) != BL_OK) return st;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    const int64_t chunk = attn_chunk(L, kv_heads, info.sms);
+    const int64_t splits = (L + chunk - 1) / chunk;
+    *bytes = (size_t)(splits * q_heads * (head_dim + 2) * 4);
+    return BL_OK;
+}
+
+bl_status bitlinear_attn_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                                int64_t L, int64_t q_heads, int64_t kv_heads, int64_t head_dim,
+                                float scale, uint16_t* out, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+    bl_status st;
+    if ((st = attn_check(L, q_heads, kv_heads, head_dim)) != BL_OK) return st;
+    if (!std::isfinite(scale)) return BL_ERR_SHAPE;
+    if (!q || !k_cache || !v_cache || !out) return BL_ERR_NULL;
+    if (!aligned16(k_cache) || !aligned16(v_cache)) return BL_ERR_ALIGN;
+    int dev;
+    DeviceInfo info;
+    if ((st = current_device(&dev, &info)) != BL_OK) return st;
+    const int64_t chunk = attn_chunk(L, kv_heads, info.sms);
+    const int64_t splits = (L + chunk - 1) / chunk;
+    const size_t need = (size_t)(splits * q_heads * (head_dim + 2) * 4);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return BL_ERR_WORKSPACE;
+    AttnArgs a = {};
+    a.q = q;
+    a.k = k_cache;
+    a.v = v_cache;
+    a.part = static_cast<float*>(workspace);
+    a.L = (int)L;
+    a.kv_heads = (int)kv_heads;
+    a.chunk = (int)chunk;
+    a.qscale = scale * kLog2e;
+    const int group = (int)(q_heads / kv_heads);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return head_dim == 128 ? attn_launch_d<128>(a, group, splits, q_heads, out, s)
+                           : attn_launch_d<64>(a, group, splits, q_heads, out, s);
 }
 
 bl_status bitlinear_device_status(void* stream) {

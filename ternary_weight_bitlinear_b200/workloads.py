@@ -142,3 +142,32 @@ def config5_layer(layer, H=HIDDEN, I=INTERMEDIATE):
                 W_down=master_weights(H, I, master_seed(layer, "down")),
                 g_in=gain(H, 1000 * (layer + 1) + 10),
                 g_sub=gain(I, 1000 * (layer + 1) + 11))
+
+
+# ---------------------------------------------------------------------------
+# attention block of the decoder layer (20 query heads, 5 key/value heads of 128)
+# ---------------------------------------------------------------------------
+Q_HEADS = 20
+KV_HEADS = 5
+HEAD_DIM = 128
+MAX_POSITIONS = 2048
+
+
+def attention_decode_inputs(L, seed, q_heads=Q_HEADS, kv_heads=KV_HEADS, head_dim=HEAD_DIM,
+                            q_std=1.0):
+    """One decode token over an L-position cache: q [q_heads * head_dim] ~
+    N(0, q_std^2), k_cache and v_cache [L, kv_heads, head_dim] ~ N(0, 1), all
+    bf16 bits (seed, seed + 1, seed + 2)."""
+    q = np.random.default_rng(seed).standard_normal(q_heads * head_dim).astype(np.float32)
+    k = np.random.default_rng(seed + 1).standard_normal((L, kv_heads, head_dim)).astype(np.float32)
+    v = np.random.default_rng(seed + 2).standard_normal((L, kv_heads, head_dim)).astype(np.float32)
+    return to_bf16_bits(q * np.float32(q_std)), to_bf16_bits(k), to_bf16_bits(v)
+
+
+def rope_positions(M, seed, max_pos=MAX_POSITIONS):
+    """M token positions in [0, max_pos), the first 0 and the last max_pos - 1."""
+    p = np.random.default_rng(seed).integers(0, max_pos, M).astype(np.int32)
+    p[0] = 0
+    if M > 1:
+        p[-1] = max_pos - 1
+    return p

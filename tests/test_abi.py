@@ -272,3 +272,31 @@ def test_decode_chain_argument_checks(L):
     steps[1].p[0].P = 0x10001
     assert L.bitlinear_decode_chain_prepare(steps, 2, ws, big) == 3
     assert L.bitlinear_decode_chain_run(ws, 16, 2, None) == 5
+
+
+def test_rope_and_attention_argument_checks(L):
+    # RoPE: shape and theta are checked first, then pointers
+    assert L.bitlinear_rope(P16, P16, -1, 20, 128, 10000.0, P16, NULL) == 2
+    assert L.bitlinear_rope(P16, P16, 1, 20, 127, 10000.0, P16, NULL) == 2   # odd head_dim
+    assert L.bitlinear_rope(P16, P16, 1, 20, 2048, 10000.0, P16, NULL) == 2  # > 1024
+    assert L.bitlinear_rope(P16, P16, 1, 20, 128, 0.0, P16, NULL) == 2
+    assert L.bitlinear_rope(P16, P16, 1, 20, 128, float("inf"), P16, NULL) == 2
+    assert L.bitlinear_rope(NULL, NULL, 0, 20, 128, 10000.0, NULL, NULL) == 0  # M == 0
+    assert L.bitlinear_rope(NULL, P16, 1, 20, 128, 10000.0, P16, NULL) == 1
+    # attention: shapes before pointers and device
+    sz = ctypes.c_size_t()
+    assert L.bitlinear_attn_decode_workspace_size(0, 20, 5, 128, ctypes.byref(sz)) == 2
+    assert L.bitlinear_attn_decode_workspace_size(16, 20, 6, 128, ctypes.byref(sz)) == 2  # 20 % 6
+    assert L.bitlinear_attn_decode_workspace_size(16, 48, 3, 128, ctypes.byref(sz)) == 2  # group 16
+    assert L.bitlinear_attn_decode_workspace_size(16, 20, 5, 96, ctypes.byref(sz)) == 2
+    assert L.bitlinear_attn_decode_workspace_size(16, 20, 5, 128, None) == 1
+    a = [P16, P16, P16]
+    assert L.bitlinear_attn_decode(*a, 0, 20, 5, 128, 0.088, P16, P16, 1 << 20, NULL) == 2
+    assert L.bitlinear_attn_decode(*a, 16, 20, 5, 128, float("nan"), P16, P16, 1 << 20, NULL) == 2
+    assert L.bitlinear_attn_decode(P16, NULL, P16, 16, 20, 5, 128, 0.088, P16, P16, 1 << 20, NULL) == 1
+    assert L.bitlinear_attn_decode(P16, P17, P16, 16, 20, 5, 128, 0.088, P16, P16, 1 << 20, NULL) == 3
+
+
+def test_binding_exports_attention_block():
+    for name in ("bitlinear_rope", "bitlinear_attn_decode", "bitlinear_attn_decode_workspace_size"):
+        assert callable(getattr(B, name))
