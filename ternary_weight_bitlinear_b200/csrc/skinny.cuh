@@ -324,18 +324,6 @@ __device__ __forceinline__ void sk_store(const SkProblem& pr, int m, int64_t n, 
     }
 }
 
-// One output of a gate/up pair: relu2_mul(bf16 gate, bf16 up), both rescaled
-// through the token's reciprocal, each with its own weight scale.
-__device__ __forceinline__ void sk_store_gate_up(const SkProblem& pr, int m, int64_t n, int acc_g,
-                                                 int acc_u, float s_x, float s_rcp) {
-    const bool sfast = s_x >= 0x1p-40f && s_x <= 0x1p40f;
-    const bool fg = sfast && pr.beta >= 0x1p-40f && pr.beta <= 0x1p40f;
-    const bool fu = sfast && pr.beta2 >= 0x1p-40f && pr.beta2 <= 0x1p40f;
-    const uint16_t a = float_to_bf16_bits(sk_scale(acc_g, pr.beta, PairDiv{s_x, s_rcp, -s_x, fg}));
-    const uint16_t bb = float_to_bf16_bits(sk_scale(acc_u, pr.beta2, PairDiv{s_x, s_rcp, -s_x, fu}));
-    static_cast<uint16_t*>(pr.y)[(int64_t)m * pr.N + n] = relu2_mul_one(a, bb);
-}
-
 template <int EW>
 __global__ void __launch_bounds__(sk_threads(EW), 1) skinny_tc_kernel(const __grid_constant__ SkBatch b) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -634,16 +622,21 @@ __global__ void __launch_bounds__(sk_threads(EW), 1) skinny_tc_kernel(const __gr
                     tmem_ld8_nowait(taddr + (uint32_t)cg, v8);
                     tmem_ld_wait();
                     if (pr.epi == kEpiGateUp) {
-                        // the up row of bit pair bit + 2 sits 16 lanes up
-                        uint32_t u8[8];
+                        // every lane rescales its own row (gate rows: bit pairs 0, 1
+                        // with the gate's scale; up rows: 2, 3 with the up's), then
+                        // the up value moves 16 lanes down to its gate row
+                        const float bl = bit < 2 ? pr.beta : pr.beta2;
+                        const bool bok = bl >= 0x1p-40f && bl <= 0x1p40f;
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) u8[k] = __shfl_down_sync(0xffffffffu, v8[k], 16);
-                        if (bit < 2 && r < pr.R) {
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                if (cg + k < cend)
-                                    sk_store_gate_up(pr, cg + k, n, (int)v8[k] - tok_rs[cg + k],
-                                                     (int)u8[k] - tok_rs[cg + k], tok_s[cg + k], tok_y[cg + k]);
+                        for (int k = 0; k < 8; ++k) {
+                            const float sx = tok_s[cg + k];
+                            const bool fast = bok && sx >= 0x1p-40f && sx <= 0x1p40f;
+                            const uint16_t mine = float_to_bf16_bits(
+                                sk_scale((int)v8[k] - tok_rs[cg + k], bl, PairDiv{sx, tok_y[cg + k], -sx, fast}));
+                            const uint32_t up = __shfl_down_sync(0xffffffffu, (uint32_t)mine, 16);
+                            if (bit < 2 && r < pr.R && cg + k < cend)
+                                static_cast<uint16_t*>(pr.y)[(int64_t)(cg + k) * pr.N + n] =
+                                    relu2_mul_one(mine, up);
                         }
                     } else if (r < pr.R) {
 #pragma unroll
