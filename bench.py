@@ -590,6 +590,77 @@ class DecodeChainWorkload:
             B.bitlinear_act_quant(self.z, L["gs"], eps, q=self.qs, s_x=self.sv[2], rowsum=self.rv[2])
             B.bitlinear_forward_quantized_batch(L["down"], 1)
 
+    def with_attention(self, dec, L=1024):
+        """The full dependent decode step of the 2B4T decoder layer: per layer
+        the input norm + q|k|v (k and v written straight into row L - 1 of the
+        layer's key/value cache), RoPE of q and of that key row, grouped-query
+        attention over the L cached positions, attn_sub_norm + o + residual,
+        then the FFN block as above.  Twelve launches a layer; the caches hold
+        seeded random keys and values for the L - 1 earlier positions."""
+        B, WL = self.B, self.WL
+        byname = {(q["layer"], q["name"]): q for q in dec.problems}
+        H, Hq, Hkv, d = WL.HIDDEN, WL.Q_HEADS, WL.KV_HEADS, WL.HEAD_DIM
+        dev = "cuda"
+        self.L_att = L
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+        self.qbuf = torch.empty((1, H), dtype=torch.bfloat16, device=dev)
+        self.att = torch.empty(H, dtype=torch.bfloat16, device=dev)
+        self.qo = torch.empty((1, H), dtype=torch.int8, device=dev)
+        self.svo = torch.empty(1, dtype=torch.float32, device=dev)
+        self.rvo = torch.empty(1, dtype=torch.int32, device=dev)
+        self.pos = torch.full((1,), L - 1, dtype=torch.int32, device=dev)
+        self.att_ws = torch.empty(max(16, B.bitlinear_attn_decode_workspace_size(L, Hq, Hkv, d)),
+                                  dtype=torch.uint8, device=dev)
+        self.kv_bytes = 0
+        for l, Lr in enumerate(self.layers):
+            _, k0, v0 = WL.attention_decode_inputs(L, seed=5000 + 10 * l)
+            Lr["kc"], Lr["vc"] = bf(k0), bf(v0)
+            krow, vrow = Lr["kc"][L - 1].reshape(1, Hkv * d), Lr["vc"][L - 1].reshape(1, Hkv * d)
+            Lr["krow"] = krow
+            Lr["gsub"] = torch.from_numpy(WL.gain(H, 1000 * (l + 1) + 13).view(np.int16)).view(
+                torch.bfloat16).cuda()
+            Lr["qkv_att"] = B.make_quantized_batch([
+                dict(q=self.qa, s_x=self.sv[0], rowsum=self.rv[0], P=byname[(l, n)]["P"],
+                     beta=byname[(l, n)]["beta"], y=y)
+                for n, y in zip(("q", "k", "v"), (self.qbuf, krow, vrow))])
+            Lr["o_att"] = B.make_quantized_batch([
+                dict(q=self.qo, s_x=self.svo, rowsum=self.rvo, P=byname[(l, "o")]["P"],
+                     beta=byname[(l, "o")]["beta"], y=self.x, residual=self.x)])
+            self.kv_bytes += L * Hkv * d * 2 * 2
+        self.att_scale = 1.0 / math.sqrt(d)
+        self.agraph = capture_graph(self.run_attention)
+
+    def run_attention(self):
+        B, WL, eps = self.B, self.WL, self.WL.RMS_EPS
+        self.x.copy_(self.x0)
+        for Lr in self.layers:
+            B.bitlinear_act_quant(self.x, Lr["ga"], eps, q=self.qa, s_x=self.sv[0], rowsum=self.rv[0])
+            B.bitlinear_forward_quantized_batch(Lr["qkv_att"], 1)
+            B.bitlinear_rope(self.qbuf, self.pos, WL.Q_HEADS, 500000.0, out=self.qbuf)
+            B.bitlinear_rope(Lr["krow"], self.pos, WL.KV_HEADS, 500000.0, out=Lr["krow"])
+            B.bitlinear_attn_decode(self.qbuf.reshape(-1), Lr["kc"], Lr["vc"], self.L_att, WL.Q_HEADS,
+                                    WL.KV_HEADS, self.att_scale, out=self.att, workspace=self.att_ws)
+            B.bitlinear_act_quant(self.att.reshape(1, -1), Lr["gsub"], eps, q=self.qo, s_x=self.svo,
+                                  rowsum=self.rvo)
+            B.bitlinear_forward_quantized_batch(Lr["o_att"], 1)
+            B.bitlinear_act_quant(self.x, Lr["gf"], eps, q=self.qf, s_x=self.sv[1], rowsum=self.rv[1])
+            B.bitlinear_forward_gate_up(self.qf, self.sv[1], self.rv[1], Lr["P2"], Lr["bg"], Lr["bu"],
+                                        out=self.z)
+            B.bitlinear_act_quant(self.z, Lr["gs"], eps, q=self.qs, s_x=self.sv[2], rowsum=self.rv[2])
+            B.bitlinear_forward_quantized_batch(Lr["down"], 1)
+
+    def measure_attention(self, reps, warmup, world, hbm):
+        ms = timed(self.agraph.replay, reps, warmup, world) / reps
+        tot = self.weight_bytes + self.kv_bytes
+        gbs = tot / (ms / 1000.0) / 1e9
+        return {"workload": "full dependent decode step: one token through the %d BitNet-2B4T "
+                            "layers in order, each norm + q|k|v, RoPE, GQA attention over a "
+                            "%d-position cache, attn_sub_norm + o + residual, then the FFN block"
+                            % (len(self.layers), self.L_att),
+                "token_us": ms * 1000.0, "tokens_per_s": job_throughput(1, world, ms),
+                "bytes": tot, "gbs": gbs, "frac_of_hbm": gbs / hbm, "reps": reps,
+                "launches_per_step": 12 * len(self.layers)}
+
     def persistent(self, dec):
         """The same token's steps as one persistent launch (3 steps a layer:
         q|k|v + o, gate|up, down), on a second pair of residual buffers."""
@@ -1050,6 +1121,8 @@ def main():
         legs["decode_chain"] = dc.measure(reps, rw, world, hbm)
         dc.persistent(wl)
         legs["decode_chain_persistent"] = dc.measure_persistent(reps, rw, world, hbm)
+        dc.with_attention(wl)
+        legs["decode_step_with_attention"] = dc.measure_attention(reps, rw, world, hbm)
         del dc
     if not args.no_skinny:
         att = {"workload": "attention block of one decode token, 2B4T heads (20 query, 5 key/value "
