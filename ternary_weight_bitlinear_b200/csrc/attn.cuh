@@ -20,9 +20,10 @@
 //  * Decode attention, split over the cache (one query token is far too
 //    little work for one CTA per head): CTA (split, kv head) takes a chunk of
 //    positions and all query heads of the group, so each key and value row
-//    is read once for the group.  A lane scores one position against every
-//    head of the group (the row's 16-byte vectors against the group's queries,
-//    pre-scaled by scale * log2(e), in shared memory), the warp keeps an
+//    is read once for the group.  Four lanes score one position against every
+//    head of the group (a quarter of the key row each against the group's
+//    queries, pre-scaled by scale * log2(e), in shared memory; two shuffles
+//    finish the dot products), eight positions a warp pass; the warp keeps an
 //    online softmax per head (running max, sum, and output vector: a lane
 //    holds d/32 dimensions, the value rows read coalesced by the warp), and
 //    the CTA merges its warps into one partial (max, sum, vector) per head in
@@ -37,7 +38,8 @@
 
 namespace bl {
 
-constexpr int kAttnThreads = 64;   // two warps a CTA, 32 positions each per pass
+constexpr int kAttnThreads = 128;  // four warps a CTA
+constexpr int kAttnPos = 8;        // positions a warp scores per pass (four lanes each)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // y[m, h d + i], y[m, h d + i + d/2] for the pair of thread i of (head h, token m).
@@ -84,10 +86,14 @@ __device__ __forceinline__ float warp_sum_f(float v) {
 }
 
 // One split of one key/value head: its NR query heads over positions
-// [sp * chunk, min(L, (sp + 1) * chunk)).
+// [sp * chunk, min(L, (sp + 1) * chunk)).  A warp takes 8 positions a pass:
+// four lanes per position each score a quarter of the head dimension (then
+// two shuffles complete the dot products), and each lane accumulates D/32
+// output dimensions of the 8 value rows.
 template <int D, int NR>
 __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnArgs a) {
-    constexpr int DL = D / 32;  // output dimensions per lane
+    constexpr int DL = D / 32;      // output dimensions per lane
+    constexpr int DP = D / 4;       // score dimensions per lane (a quarter of the head)
     constexpr int NW = kAttnThreads / 32;
     __shared__ float qs[NR][D];
     __shared__ float wm[NW][NR], wl[NW][NR];
@@ -95,6 +101,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnArgs
     const int g = blockIdx.y, sp = blockIdx.x;
     const int H = a.kv_heads * NR;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int jl = lane >> 2, part = lane & 3;  // this lane's position in the pass, quarter of the head
     const int j0 = sp * a.chunk, j1 = min(a.L, j0 + a.chunk);
     pdl_wait();
     pdl_launch_dependents();
@@ -111,23 +118,23 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnArgs
         for (int e = 0; e < DL; ++e) o[h][e] = 0.0f;
     }
     const int64_t row_stride = (int64_t)a.kv_heads * D;  // elements between positions
-    for (int jb = j0 + 32 * warp; jb < j1; jb += 32 * NW) {
-        // every load of the pass in flight at once: this lane's key row, and
-        // its DL dimensions of the warp's 32 value rows (values do not depend
-        // on the scores)
-        const int j = jb + lane;
-        const int nj = min(32, j1 - jb);
-        uint4 kr[D / 8];
-        if (j < j1) {
-            const uint4* kp = reinterpret_cast<const uint4*>(a.k + (int64_t)j * row_stride + (int64_t)g * D);
+    for (int jb = j0 + kAttnPos * warp; jb < j1; jb += kAttnPos * NW) {
+        // every load of the pass in flight at once: this lane's quarter of its
+        // position's key row, and its D/32 dimensions of the pass's value rows
+        const int j = jb + jl;
+        const bool valid = j < j1;
+        uint4 kr[DP / 8];
+        if (valid) {
+            const uint4* kp =
+                reinterpret_cast<const uint4*>(a.k + (int64_t)j * row_stride + (int64_t)g * D + part * DP);
 #pragma unroll
-            for (int c = 0; c < D / 8; ++c) kr[c] = __ldcg(kp + c);
+            for (int c = 0; c < DP / 8; ++c) kr[c] = __ldcg(kp + c);
         }
-        uint32_t vr[32][DL / 2];
+        uint32_t vr[kAttnPos][DL / 2];
         const uint16_t* vbase = a.v + (int64_t)jb * row_stride + (int64_t)g * D + lane * DL;
 #pragma unroll
-        for (int b = 0; b < 32; ++b) {
-            if (b < nj) {  // warp-uniform
+        for (int b = 0; b < kAttnPos; ++b) {
+            if (jb + b < j1) {  // warp-uniform
                 const uint16_t* vp = vbase + (int64_t)b * row_stride;
                 if constexpr (DL == 4) {
                     const uint2 vv = __ldcg(reinterpret_cast<const uint2*>(vp));
@@ -141,44 +148,47 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnArgs
                 for (int e = 0; e < DL / 2; ++e) vr[b][e] = 0u;
             }
         }
-        // scores of this lane's position against the group's heads (log2 domain)
+        // scores (log2 domain): a quarter dot product per lane, then the four lanes' sum
         float s[NR];
 #pragma unroll
         for (int h = 0; h < NR; ++h) s[h] = 0.0f;
-        if (j < j1) {
+        if (valid) {
 #pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-                const uint4 kv = kr[c];
-                const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
+            for (int c = 0; c < DP / 8; ++c) {
+                const uint32_t w[4] = {kr[c].x, kr[c].y, kr[c].z, kr[c].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float k0 = bf16_bits_to_float(w[e] & 0xFFFFu), k1 = bf16_bits_to_float(w[e] >> 16);
+                    const int dd = part * DP + 8 * c + 2 * e;
 #pragma unroll
                     for (int h = 0; h < NR; ++h) {
-                        s[h] = fmaf(k0, qs[h][8 * c + 2 * e], s[h]);
-                        s[h] = fmaf(k1, qs[h][8 * c + 2 * e + 1], s[h]);
+                        s[h] = fmaf(k0, qs[h][dd], s[h]);
+                        s[h] = fmaf(k1, qs[h][dd + 1], s[h]);
                     }
                 }
             }
-        } else {
-#pragma unroll
-            for (int h = 0; h < NR; ++h) s[h] = -INFINITY;
         }
-        // online softmax over these 32 positions (lane 0's position is valid)
+#pragma unroll
+        for (int h = 0; h < NR; ++h) {
+            s[h] += __shfl_xor_sync(0xffffffffu, s[h], 1);
+            s[h] += __shfl_xor_sync(0xffffffffu, s[h], 2);
+            if (!valid) s[h] = -INFINITY;
+        }
+        // online softmax over the pass's positions (position jb is valid)
         float p[NR];
 #pragma unroll
         for (int h = 0; h < NR; ++h) {
             const float mn = fmaxf(m[h], warp_max_f(s[h]));
-            const float alpha = exp2f(m[h] - mn);  // 0 on the first block (m = -inf)
+            const float alpha = exp2f(m[h] - mn);  // 0 on the first pass (m = -inf)
             p[h] = exp2f(s[h] - mn);               // 0 for positions past the chunk
-            l[h] = fmaf(l[h], alpha, warp_sum_f(p[h]));
+            l[h] = fmaf(l[h], alpha, warp_sum_f(part == 0 ? p[h] : 0.0f));
 #pragma unroll
             for (int e = 0; e < DL; ++e) o[h][e] *= alpha;
             m[h] = mn;
         }
-        // weighted values (rows past nj are zeros with weight 0)
+        // weighted values (rows past the chunk are zeros with weight 0)
 #pragma unroll
-        for (int b = 0; b < 32; ++b) {
+        for (int b = 0; b < kAttnPos; ++b) {
             float vf[DL];
 #pragma unroll
             for (int e = 0; e < DL / 2; ++e) {
@@ -187,7 +197,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnArgs
             }
 #pragma unroll
             for (int h = 0; h < NR; ++h) {
-                const float pj = __shfl_sync(0xffffffffu, p[h], b);
+                const float pj = __shfl_sync(0xffffffffu, p[h], 4 * b);
 #pragma unroll
                 for (int e = 0; e < DL; ++e) o[h][e] = fmaf(pj, vf[e], o[h][e]);
             }

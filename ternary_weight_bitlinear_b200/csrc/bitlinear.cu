@@ -753,7 +753,8 @@ bl_status forward_impl(const uint16_t* x, const uint16_t* gain, float eps, const
 namespace {
 
 // Positions per split: enough splits for two CTAs per SM over the key/value
-// heads, at least 32 positions (one warp's block) each.
+// heads, at least 32 positions (one pass of the CTA's four warps) each; more
+// splits make the merge, which reads every split's partial, the longer part.
 int64_t attn_chunk(int64_t L, int64_t kv_heads, int sms) {
     const int64_t target = std::max<int64_t>(1, (2 * (int64_t)sms + kv_heads - 1) / kv_heads);
     const int64_t per = (L + target - 1) / target;
