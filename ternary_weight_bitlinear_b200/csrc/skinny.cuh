@@ -588,18 +588,53 @@ __global__ void __launch_bounds__(sk_threads(EW), 1) skinny_tc_kernel(const __gr
                 write = lf == 1u;
                 if (write) {
                     __threadfence();
-                    for (int64_t c2 = cf; c2 <= cl; ++c2) {
-                        if (c2 == c) continue;
-                        const int32_t* other =
-                            b.part + ((size_t)(2 * c2 + (c2 == cf ? 1 : 0)) * 128 + row128) * b.npad;
+                    auto other_part = [&](int64_t c2) {
+                        return b.part + ((size_t)(2 * c2 + (c2 == cf ? 1 : 0)) * 128 + row128) * b.npad;
+                    };
+                    if constexpr (EW == 4) {
+                        // the others' partial sums, two participants' loads in flight
+                        // at a time (a participant's sums are one L2 round trip)
+                        int64_t c2 = cf == c ? cf + 1 : cf;
+                        while (c2 <= cl) {
+                            int64_t c3 = c2 + 1;
+                            if (c3 == c) ++c3;
+                            const int32_t* o2 = other_part(c2);
+                            const int32_t* o3 = other_part(c3 <= cl ? c3 : c2);
+                            // four epilogue warps serve npad 16: 16 columns a thread
+                            uint4 w2[4], w3[4];
 #pragma unroll
-                        for (int k = 0; k < 32; k += 4) {
-                            if (c0 + k < c1) {
-                                const uint4 w4 = __ldcg(reinterpret_cast<const uint4*>(other + c0 + k));
-                                v[k] += w4.x;
-                                v[k + 1] += w4.y;
-                                v[k + 2] += w4.z;
-                                v[k + 3] += w4.w;
+                            for (int k = 0; k < 16; k += 4) {
+                                if (c0 + k < c1) {
+                                    w2[k / 4] = __ldcg(reinterpret_cast<const uint4*>(o2 + c0 + k));
+                                    w3[k / 4] = c3 <= cl ? __ldcg(reinterpret_cast<const uint4*>(o3 + c0 + k))
+                                                         : make_uint4(0u, 0u, 0u, 0u);
+                                }
+                            }
+#pragma unroll
+                            for (int k = 0; k < 16; k += 4) {
+                                if (c0 + k < c1) {
+                                    v[k] += w2[k / 4].x + w3[k / 4].x;
+                                    v[k + 1] += w2[k / 4].y + w3[k / 4].y;
+                                    v[k + 2] += w2[k / 4].z + w3[k / 4].z;
+                                    v[k + 3] += w2[k / 4].w + w3[k / 4].w;
+                                }
+                            }
+                            c2 = c3 + 1;
+                            if (c2 == c) ++c2;
+                        }
+                    } else {
+                        for (int64_t c2 = cf; c2 <= cl; ++c2) {
+                            if (c2 == c) continue;
+                            const int32_t* other = other_part(c2);
+#pragma unroll
+                            for (int k = 0; k < 32; k += 4) {
+                                if (c0 + k < c1) {
+                                    const uint4 w4 = __ldcg(reinterpret_cast<const uint4*>(other + c0 + k));
+                                    v[k] += w4.x;
+                                    v[k + 1] += w4.y;
+                                    v[k + 2] += w4.z;
+                                    v[k + 3] += w4.w;
+                                }
                             }
                         }
                     }
