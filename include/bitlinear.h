@@ -383,7 +383,7 @@ bl_status bitlinear_decode_chain_run(void* workspace, size_t workspace_bytes, in
  *   Scratch: instead of a caller workspace it uses one file-scope device array
  *   of BL_NOALLOC_SCRATCH_BYTES that every GPU which loads the library keeps
  *   until the process exits.  The first call on a device looks up that array's
- *   device address (so make that first call before any stream capture).
+ *   device address with a host-side runtime query.
  *   The array must hold the int8 codes, scales and row sums of the input
  *   (M*K bytes plus 8*M, each part rounded up to 256 bytes); larger shapes are
  *   rejected with BL_ERR_WORKSPACE before anything is launched, and
